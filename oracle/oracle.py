@@ -1,0 +1,335 @@
+"""Plain fp64 CPU oracle for dynamic tile-sparse global attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+benchmark's CPU-baseline / reference arm may import this module; the product
+path (the C-ABI library and its Python binding) never does, and there is no
+CPU fallback built on it.  It shares no code with the CUDA path: it reads the
+same seeded inputs (bf16 bit patterns or float32), converts them exactly to
+float64 and recomputes every step with numpy in the order the method states.
+
+The method (what is computed, and where each step comes from):
+
+* Global (cross-frame) attention in VGGT-style backbones: every query token of
+  every one of S frames attends to all S*N tokens, at quadratic cost in the
+  number of frames ("AVGGT: Rethinking Global Attention for Accelerating VGGT",
+  technical summary, section 1 "O Problema"; "(Full) Attention is More Than
+  You Need", the full-vs-sparse figure).
+* Dynamic sparsity: keep only the most promising query-key interactions,
+  chosen per input, per layer and per head ("SAF3R: Dynamic Sparse Attention
+  for Feed-Forward 3D Reconstruction Transformers", abstract).  The generic
+  mechanism used here is tile-sparse attention ("Zebra3D: Efficient Hybrid
+  Foundation Models For Scalable 3D Reconstruction", abstract): tiles of
+  queries and keys are summarised by their means, scored by a per-head dot
+  product, and each query tile keeps its top-k key tiles.
+* Kept always: the query's own frame (frame attention is the cheap local
+  case, AVGGT section 2.B.1, and the diagonal/self term is preserved, AVGGT
+  section 2.B.2 "Preservacao Diagonal") and the special camera/register
+  tokens of every frame (AVGGT section 2.B.2: all queries and special tokens
+  are kept).
+* Landmarks: unselected key tiles are not dropped but summarised (Zebra3D
+  abstract, "landmark summaries to preserve unselected context"; AVGGT
+  section 2.B.2 approximates discarded columns by a mean key/value pair).
+  Each unselected tile j contributes one token (mean K, mean V) whose logit
+  carries +ln(c_j), c_j the number of key rows it stands for, so that it
+  weighs as c_j copies of the mean key.
+
+Readings taken where the pages are silent (all listed in the design notes):
+tiles are frame aligned (the last tile of a frame is partial); k counts only
+tiles outside the own frame; sink keys are excluded from tiles and attended
+exactly once each; sink rows are ordinary queries; the score is the plain dot
+product of fp64 tile means (no 1/sqrt(d), which does not change a ranking);
+equal scores go to the lower key-tile index; the landmark bias is added after
+the softmax scale.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------- inputs
+
+def to_f64(a: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) or float32 to float64."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if a.dtype in (np.float32, np.float64):
+        return a.astype(np.float64)
+    raise TypeError("unsupported input dtype %s" % a.dtype)
+
+
+# ----------------------------------------------------------------------------- geometry
+
+@dataclasses.dataclass(frozen=True)
+class Geometry:
+    """Frame-aligned tiling of S frames x N tokens (token t = s*N + n)."""
+    frames: int
+    tokens: int
+    tile: int
+    n_sink: int
+
+    @property
+    def L(self) -> int:
+        return self.frames * self.tokens
+
+    @property
+    def tpf(self) -> int:
+        return -(-self.tokens // self.tile)
+
+    @property
+    def nt(self) -> int:
+        return self.frames * self.tpf
+
+    def frame_of_tile(self, j: int) -> int:
+        return j // self.tpf
+
+    def tile_rows(self, j: int) -> np.ndarray:
+        """All token indices of tile j (its query rows)."""
+        f, slot = divmod(j, self.tpf)
+        lo = slot * self.tile
+        hi = min(self.tokens, lo + self.tile)
+        return f * self.tokens + np.arange(lo, hi)
+
+    def tile_key_rows(self, j: int) -> np.ndarray:
+        """Token indices of tile j that enter tile visits and key pooling (non-sink)."""
+        f, slot = divmod(j, self.tpf)
+        lo = max(slot * self.tile, self.n_sink)
+        hi = min(self.tokens, slot * self.tile + self.tile)
+        if hi <= lo:
+            return np.zeros((0,), np.int64)
+        return f * self.tokens + np.arange(lo, hi)
+
+    def sink_rows(self) -> np.ndarray:
+        """Every frame's special tokens, frame-major (the sink segment order)."""
+        return np.array([s * self.tokens + n for s in range(self.frames) for n in range(self.n_sink)],
+                        dtype=np.int64)
+
+    def key_count(self, j: int) -> int:
+        """Number of non-sink rows of tile j (the landmark multiplicity c_j)."""
+        return len(self.tile_key_rows(j))
+
+    def own_frame_tiles(self, i: int) -> np.ndarray:
+        f = self.frame_of_tile(i)
+        return np.arange(f * self.tpf, (f + 1) * self.tpf)
+
+
+# ----------------------------------------------------------------------------- step 1: pooling
+
+def pool(g: Geometry, q: np.ndarray, k: np.ndarray, v: np.ndarray | None = None):
+    """Tile means (Zebra3D abstract: tiles summarised by landmarks; AVGGT 2.B.2 mean K-V pair).
+
+    q, k, v: [BH][L][d] float64.  Returns (q_bar, k_bar, v_bar, cnt, sink_k, sink_v):
+      q_bar[h, j] = mean of q over all rows of tile j;
+      k_bar[h, j] = mean of k over the non-sink rows of tile j (0 if there are none);
+      v_bar likewise (None when v is None);
+      cnt[j]      = number of non-sink rows of tile j;
+      sink_k/v    = the sink rows of every frame, frame-major, [BH][S*n_sink][d].
+    """
+    bh, L, d = q.shape
+    assert L == g.L
+    nt = g.nt
+    q_bar = np.zeros((bh, nt, d))
+    k_bar = np.zeros((bh, nt, d))
+    v_bar = None if v is None else np.zeros((bh, nt, v.shape[2]))
+    cnt = np.zeros((nt,), np.int64)
+    for j in range(nt):
+        rq = g.tile_rows(j)
+        rk = g.tile_key_rows(j)
+        q_bar[:, j] = q[:, rq].mean(axis=1)
+        cnt[j] = len(rk)
+        if len(rk):
+            k_bar[:, j] = k[:, rk].mean(axis=1)
+            if v is not None:
+                v_bar[:, j] = v[:, rk].mean(axis=1)
+    sr = g.sink_rows()
+    sink_k = k[:, sr]
+    sink_v = None if v is None else v[:, sr]
+    return q_bar, k_bar, v_bar, cnt, sink_k, sink_v
+
+
+# ----------------------------------------------------------------------------- step 2: scores
+
+def scores(q_bar: np.ndarray, k_bar: np.ndarray) -> np.ndarray:
+    """Per-head tile scores s[h, i, j] = q_bar[h, i] . k_bar[h, j] (SAF3R abstract: rank the
+    query-key interactions by promise; the dot product of tile means is the ranking signal)."""
+    return np.einsum("hid,hjd->hij", q_bar, k_bar)
+
+
+# ----------------------------------------------------------------------------- step 3: selection
+
+def candidates(g: Geometry, i: int) -> np.ndarray:
+    """Key tiles that query tile i may choose: outside its own frame, with a non-sink row."""
+    forced = g.own_frame_tiles(i)
+    cand = np.setdiff1d(np.arange(g.nt), forced)
+    return np.array([j for j in cand if g.key_count(int(j)) > 0], dtype=np.int64)
+
+
+def select_row(g: Geometry, s_row: np.ndarray, i: int, k: int) -> np.ndarray:
+    """Kept key tiles of query tile i, ascending.
+
+    Forced: every tile of the query's own frame (AVGGT 2.B.1 frame attention and the preserved
+    diagonal of 2.B.2).  Chosen: the k highest-scoring tiles among the candidates, ordered by
+    (score descending, index ascending); all of them when k >= their number.
+    """
+    forced = g.own_frame_tiles(i)
+    cand = candidates(g, i)
+    kk = max(0, min(int(k), len(cand)))
+    order = np.lexsort((cand, -s_row[cand]))  # primary: -score, secondary: index
+    chosen = cand[order[:kk]]
+    return np.sort(np.concatenate([forced, chosen]))
+
+
+def select(g: Geometry, s: np.ndarray, k: int):
+    """kept[h][i] for every head h and query tile i."""
+    bh = s.shape[0]
+    return [[select_row(g, s[h, i], i, k) for i in range(g.nt)] for h in range(bh)]
+
+
+def max_kept(g: Geometry, k: int) -> int:
+    """Length of every kept list: own-frame tiles plus min(k, candidates)."""
+    n_cand = (g.frames - 1) * sum(1 for slot in range(g.tpf) if g.key_count(slot) > 0)
+    return g.tpf + max(0, min(int(k), n_cand))
+
+
+# ----------------------------------------------------------------------------- step 4: attention
+
+def _softmax_rows(logits: np.ndarray, values: np.ndarray):
+    """Two-pass softmax of each row of `logits` applied to `values`; returns (O, LSE)."""
+    m = logits.max(axis=1, keepdims=True)
+    w = np.exp(logits - m)
+    z = w.sum(axis=1, keepdims=True)
+    o = (w @ values) / z
+    lse = (m + np.log(z))[:, 0]
+    return o, lse
+
+
+def attend_tile(g: Geometry, q: np.ndarray, k: np.ndarray, v: np.ndarray, h: int, i: int,
+                kept: np.ndarray, scale: float, landmark: bool = False,
+                k_bar: np.ndarray | None = None, v_bar: np.ndarray | None = None,
+                cnt: np.ndarray | None = None):
+    """Outputs of the query rows of tile i of head h on a given kept list.
+
+    Attended set of every row (Zebra3D abstract; AVGGT 2.B.2):
+      (i)   the non-sink rows of every listed tile,
+      (ii)  every frame's sink rows, once each,
+      (iii) in landmark mode, one token (k_bar_j, v_bar_j) with logit bias ln(cnt_j)
+            for every unlisted tile j with cnt_j > 0.
+    Logits are scale * q.k (+ bias); softmax is taken over the whole attended set.
+    """
+    rows = g.tile_rows(i)
+    key_rows = [g.tile_key_rows(int(j)) for j in kept]
+    key_rows.append(g.sink_rows())
+    kr = np.concatenate(key_rows) if key_rows else np.zeros((0,), np.int64)
+    qh = q[h, rows]
+    logits = scale * (qh @ k[h, kr].T)
+    values = v[h, kr]
+    if landmark:
+        listed = np.zeros((g.nt,), bool)
+        listed[np.asarray(kept, np.int64)] = True
+        lm = np.nonzero((~listed) & (cnt > 0))[0]
+        if len(lm):
+            lm_logits = scale * (qh @ k_bar[h, lm].T) + np.log(cnt[lm].astype(np.float64))[None, :]
+            logits = np.concatenate([logits, lm_logits], axis=1)
+            values = np.concatenate([values, v_bar[h, lm]], axis=0)
+    return rows, _softmax_rows(logits, values)
+
+
+def attend(g: Geometry, q: np.ndarray, k: np.ndarray, v: np.ndarray, kept, scale: float,
+           landmark: bool = False, k_bar=None, v_bar=None, cnt=None, items=None):
+    """Full output O [BH][L][d] and LSE [BH][L] (NaN where a row was not computed).
+
+    `kept[h][i]` is the list for query tile i of head h; `items`, if given, restricts the
+    work to those (h, i) pairs.
+    """
+    bh, L, _ = q.shape
+    O = np.full((bh, L, v.shape[2]), np.nan)
+    LSE = np.full((bh, L), np.nan)
+    todo = items if items is not None else [(h, i) for h in range(bh) for i in range(g.nt)]
+    for h, i in todo:
+        rows, (o, lse) = attend_tile(g, q, k, v, h, i, kept[h][i], scale, landmark, k_bar, v_bar, cnt)
+        O[h, rows] = o
+        LSE[h, rows] = lse
+    return O, LSE
+
+
+def attend_bruteforce(g: Geometry, q, k, v, kept, scale: float, landmark: bool = False,
+                      k_bar=None, v_bar=None, cnt=None):
+    """Same outputs as `attend`, built as one explicit [L x (L + nt)] bias matrix per head
+    (0 where a pair is attended, -inf where it is not, ln cnt_j on landmark columns) followed
+    by a full-row softmax.  For tiny shapes only; it shares no bookkeeping with `attend`
+    beyond the tile geometry."""
+    bh, L, _ = q.shape
+    nt = g.nt
+    O = np.zeros((bh, L, v.shape[2]))
+    LSE = np.zeros((bh, L))
+    for h in range(bh):
+        bias = np.full((L, L + nt), -np.inf)
+        for t in range(L):
+            s_t, n_t = divmod(t, g.tokens)
+            i = s_t * g.tpf + n_t // g.tile  # query tile of row t
+            listed = set(int(x) for x in kept[h][i])
+            for u in range(L):
+                s_u, n_u = divmod(u, g.tokens)
+                if n_u < g.n_sink:
+                    bias[t, u] = 0.0  # special tokens: attended once by everyone
+                    continue
+                j = s_u * g.tpf + n_u // g.tile
+                if j in listed:
+                    bias[t, u] = 0.0
+            if landmark:
+                for j in range(nt):
+                    if j not in listed and cnt[j] > 0:
+                        bias[t, L + j] = math.log(cnt[j])
+        keys = k[h] if not landmark else np.concatenate([k[h], k_bar[h]], axis=0)
+        vals = v[h] if not landmark else np.concatenate([v[h], v_bar[h]], axis=0)
+        if not landmark:
+            bias = bias[:, :L]
+        logits = scale * (q[h] @ keys.T) + bias
+        O[h], LSE[h] = _softmax_rows(logits, vals)
+    return O, LSE
+
+
+def dense(q, k, v, scale: float):
+    """Textbook dense softmax attention over all L keys (the sparsity-0 control)."""
+    bh, L, _ = q.shape
+    O = np.zeros((bh, L, v.shape[2]))
+    LSE = np.zeros((bh, L))
+    for h in range(bh):
+        O[h], LSE[h] = _softmax_rows(scale * (q[h] @ k[h].T), v[h])
+    return O, LSE
+
+
+# ----------------------------------------------------------------------------- selection parity rule
+
+def selection_matches(g: Geometry, s_row: np.ndarray, i: int, k: int, got: np.ndarray,
+                      rel: float = 1e-4, floor: float = 1e-7):
+    """Check a selected list against the oracle's for query tile i (s_row in fp64).
+
+    Accepted iff it is ascending without repeats, has the oracle's size, contains every
+    own-frame tile, and every swap against the oracle's choice is between near-equal scores:
+    for a in got\\ref and b in ref\\got, s_b - s_a <= rel*max(|s_a|,|s_b|) + floor*max|s_row|.
+    Returns (ok, message).
+    """
+    ref = select_row(g, s_row, i, k)
+    got = np.asarray(got, np.int64)
+    if len(got) != len(ref):
+        return False, "size %d != %d" % (len(got), len(ref))
+    if len(got) > 1 and not np.all(np.diff(got) > 0):
+        return False, "not strictly ascending"
+    if not np.all(np.isin(g.own_frame_tiles(i), got)):
+        return False, "own-frame tile missing"
+    if got.min(initial=0) < 0 or got.max(initial=0) >= g.nt:
+        return False, "index out of range"
+    extra = np.setdiff1d(got, ref)
+    missing = np.setdiff1d(ref, got)
+    if len(extra) == 0:
+        return True, "exact"
+    smax = float(np.abs(s_row).max())
+    for a in extra:
+        for b in missing:
+            sa, sb = float(s_row[a]), float(s_row[b])
+            if sb - sa > rel * max(abs(sa), abs(sb)) + floor * smax:
+                return False, "swap %d<->%d beyond tolerance (%.9g vs %.9g)" % (a, b, sa, sb)
+    return True, "%d near-tie swaps" % len(extra)

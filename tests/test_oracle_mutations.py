@@ -1,0 +1,157 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins catch each one.
+
+Every mutant below is a one-line slip of the kind that would silently corrupt
+parity: a dropped term, a wrong sign, a swapped index, a transposed operand.
+The pins in test_oracle_pins.py must fail for every one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import tests.test_oracle_pins as pins
+from oracle import oracle as orc
+
+PIN_TESTS = [
+    lambda: pins.test_pool_against_explicit_loops(),
+    lambda: pins.test_pool_ignores_sink_keys(),
+    lambda: pins.test_scores_closed_form(),
+    lambda: pins.test_scores_not_transposed(),
+    *[lambda s=s: pins.test_select_bruteforce_subsets(s) for s in range(3)],
+    lambda: pins.test_select_edges(),
+    lambda: pins.test_select_skips_keyless_tiles(),
+    lambda: pins.test_attention_two_key_closed_form(),
+    lambda: pins.test_attention_landmark_closed_form_weight(),
+    *[lambda l=l, n=n, k=k: pins.test_list_mode_equals_explicit_mask(l, n, k)
+      for l in (False, True) for n in (0, 1) for k in (1, 99)],
+    lambda: pins.test_all_tiles_equals_textbook_dense(2),
+    lambda: pins.test_weights_sum_to_one(True),
+    lambda: pins.test_frame_permutation_equivariance(True),
+    lambda: pins.test_landmarks_exact_when_tile_keys_are_identical(),
+    lambda: pins.test_k0_is_frame_attention_plus_sinks(),
+]
+
+
+def _some_pin_fails():
+    for t in PIN_TESTS:
+        try:
+            t()
+        except (AssertionError, ValueError, IndexError):
+            return True
+    return False
+
+
+# ---- mutants -----------------------------------------------------------------------------
+
+_pool = orc.pool
+_attend_tile = orc.attend_tile
+_select_row = orc.select_row
+_softmax_rows = orc._softmax_rows
+_tile_key_rows = orc.Geometry.tile_key_rows
+
+
+def pool_with_sinks(g, q, k, v=None):
+    qb, kb, vb, cnt, sk, sv = _pool(g, q, k, v)
+    for j in range(g.nt):  # slip: key means over all rows, sinks included
+        kb[:, j] = k[:, g.tile_rows(j)].mean(axis=1)
+    return qb, kb, vb, cnt, sk, sv
+
+
+def scores_transposed(q_bar, k_bar):
+    return np.einsum("hjd,hid->hij", q_bar, k_bar)
+
+
+def select_ties_high(g, s_row, i, k):
+    forced = g.own_frame_tiles(i)
+    cand = orc.candidates(g, i)
+    kk = max(0, min(int(k), len(cand)))
+    order = np.lexsort((-cand, -s_row[cand]))  # slip: higher index wins ties
+    return np.sort(np.concatenate([forced, cand[order[:kk]]]))
+
+
+def select_counts_own_frame(g, s_row, i, k):
+    forced = g.own_frame_tiles(i)
+    return _select_row(g, s_row, i, max(0, k - len(forced)))  # slip: k includes own frame
+
+
+def select_no_force(g, s_row, i, k):
+    cand = np.arange(g.nt)  # slip: own frame competes instead of being forced
+    order = np.lexsort((cand, -s_row[cand]))
+    return np.sort(cand[order[:orc.max_kept(g, k)]])
+
+
+def _attend_variant(bias_sign=1.0, drop_scale=False, drop_sinks=False, bias_inside_scale=False):
+    def attend_tile(g, q, k, v, h, i, kept, scale, landmark=False, k_bar=None, v_bar=None, cnt=None):
+        rows = g.tile_rows(i)
+        kr = [g.tile_key_rows(int(j)) for j in kept]
+        if not drop_sinks:
+            kr.append(g.sink_rows())
+        kr = np.concatenate(kr)
+        sc = 1.0 if drop_scale else scale
+        logits = sc * (q[h, rows] @ k[h, kr].T)
+        values = v[h, kr]
+        if landmark:
+            listed = np.zeros((g.nt,), bool)
+            listed[np.asarray(kept, np.int64)] = True
+            lm = np.nonzero((~listed) & (cnt > 0))[0]
+            if len(lm):
+                b = bias_sign * np.log(cnt[lm].astype(float))[None, :]
+                if bias_inside_scale:
+                    lml = sc * (q[h, rows] @ k_bar[h, lm].T + b)
+                else:
+                    lml = sc * (q[h, rows] @ k_bar[h, lm].T) + b
+                logits = np.concatenate([logits, lml], axis=1)
+                values = np.concatenate([values, v_bar[h, lm]], axis=0)
+        return rows, orc._softmax_rows(logits, values)
+    return attend_tile
+
+
+def softmax_lse_without_max(logits, values):
+    o, lse = _softmax_rows(logits, values)
+    m = logits.max(axis=1)
+    return o, lse - m  # slip: forgot to add the running max back
+
+
+def softmax_no_normalise(logits, values):
+    m = logits.max(axis=1, keepdims=True)
+    w = np.exp(logits - m)
+    return w @ values, (m + np.log(w.sum(axis=1, keepdims=True)))[:, 0]
+
+
+def key_rows_keep_sinks(self, j):
+    f, slot = divmod(j, self.tpf)
+    lo = slot * self.tile  # slip: sink rows stay inside tile 0 of each frame
+    hi = min(self.tokens, lo + self.tile)
+    return f * self.tokens + np.arange(lo, hi)
+
+
+MUTANTS = {
+    "pool_includes_sinks": ("pool", pool_with_sinks),
+    "scores_transposed": ("scores", scores_transposed),
+    "ties_to_higher_index": ("select_row", select_ties_high),
+    "k_counts_own_frame": ("select_row", select_counts_own_frame),
+    "own_frame_not_forced": ("select_row", select_no_force),
+    "landmark_bias_negated": ("attend_tile", _attend_variant(bias_sign=-1.0)),
+    "scale_dropped": ("attend_tile", _attend_variant(drop_scale=True)),
+    "sinks_dropped": ("attend_tile", _attend_variant(drop_sinks=True)),
+    "bias_inside_scale": ("attend_tile", _attend_variant(bias_inside_scale=True)),
+    "lse_without_max": ("_softmax_rows", softmax_lse_without_max),
+    "softmax_not_normalised": ("_softmax_rows", softmax_no_normalise),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(orc, attr, fn)
+    assert _some_pin_fails(), "mutant %s survived every pin" % name
+
+
+def test_key_rows_mutant_is_caught(monkeypatch):
+    monkeypatch.setattr(orc.Geometry, "tile_key_rows", key_rows_keep_sinks)
+    assert _some_pin_fails()
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert not _some_pin_fails()
+    assert math.isfinite(1.0)
