@@ -1,0 +1,203 @@
+/*
+ * sa.h - dynamic tile-sparse global attention for feed-forward 3-D
+ * reconstruction transformers, on B200 (sm_100a).
+ *
+ * The operation.  In VGGT-style backbones a "global" attention layer lets
+ * every query token of each of S frames attend to all S*N tokens, which costs
+ * O((S*N)^2) ("AVGGT: Rethinking Global Attention for Accelerating VGGT",
+ * technical summary, section 1; "(Full) Attention is More Than You Need",
+ * full vs sparse global attention).  The sparse layer keeps only the most
+ * promising interactions, chosen per input and per head ("SAF3R: Dynamic
+ * Sparse Attention for Feed-Forward 3D Reconstruction Transformers",
+ * abstract), at tile granularity with landmark summaries of the rest
+ * ("Zebra3D: Efficient Hybrid Foundation Models For Scalable 3D
+ * Reconstruction", abstract).  The path is four calls:
+ *
+ *   sa_tile_pool        tile means of Q and K (and V for landmarks)
+ *   sa_tile_scores      per-head tile-score matrix  s = mean(Q) . mean(K)^T
+ *   sa_select_topk      per query tile: own-frame tiles + top-k other tiles
+ *   sa_sparse_attn_fwd  block-sparse softmax attention over the kept tiles,
+ *                       every frame's special tokens, and (optionally) one
+ *                       landmark token per unselected tile
+ *
+ * plus sa_dense_attn_fwd, the dense (sparsity 0) control at the same shape.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Tokens.  t = s*N + n for frame s < S and token n < N.  Tokens n < n_sink
+ *   of every frame are the camera/register ("sink") tokens.
+ * Layout.  Q, K, V, O are contiguous [bh][S*N][head_dim] arrays of the
+ *   shape's dtype (bf16 or f32); bh folds batch and heads, which are
+ *   independent problems.
+ * Tiles.  Tiles are frame aligned: frame s has tpf = ceil(N/tile) tiles, the
+ *   last one partial; tile j covers frame j / tpf, tokens
+ *   [(j%tpf)*tile, min(N, (j%tpf+1)*tile)).  nt = S*tpf (sa_num_tiles).
+ *   A tile's KEY rows are its tokens with n >= n_sink; sink keys are never
+ *   part of a tile and are attended once by every query instead.
+ * Pointers.  Every array argument is a DEVICE pointer on the current device,
+ *   16-byte aligned and contiguous; the caller allocates and owns all of
+ *   them (the library keeps only a device error word and per-device launch
+ *   attributes).  Optional arguments are marked _or_null.
+ * Streams.  Every compute call is asynchronous on `stream` (NULL = legacy
+ *   default stream) and never synchronises, except sa_check_device_error.
+ * Errors.  Arguments are validated on the host before any launch: an invalid
+ *   shape, a NULL required pointer or a misaligned pointer returns
+ *   SA_ERR_INVALID_ARG (or SA_ERR_UNSUPPORTED for a shape outside the built
+ *   kernels) and touches no output.  A failed launch returns SA_ERR_CUDA.
+ *   Errors found on the device (a bounded wait that ran out, a kept list
+ *   with an out-of-range entry) are recorded in a device error word that
+ *   sa_check_device_error reads and clears.
+ * Threads.  Calls on different streams with disjoint outputs may run
+ *   concurrently from several host threads.
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* sa_stream_t;
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,   /* bad shape, NULL or misaligned pointer, bad size */
+    SA_ERR_UNSUPPORTED = 2,   /* valid, but outside what the built kernels handle */
+    SA_ERR_CUDA = 3,          /* a CUDA runtime/driver call or a launch failed */
+    SA_ERR_TIMEOUT = 4,       /* a device-side wait ran out of its time limit */
+    SA_ERR_BAD_LIST = 5,      /* a kept list held an index outside [0, nt) */
+    SA_ERR_WORKSPACE = 6      /* workspace NULL or smaller than the _workspace_size query */
+} sa_status;
+
+typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
+
+typedef struct {
+    int32_t bh;            /* batch * heads: independent problems (>= 1) */
+    int32_t frames;        /* S (>= 1) */
+    int32_t tokens;        /* N tokens per frame (>= 1) */
+    int32_t head_dim;      /* d; 64 is built (else SA_ERR_UNSUPPORTED) */
+    int32_t tile;          /* T in {64, 128} */
+    int32_t n_sink;        /* special tokens per frame, 0 <= n_sink < tokens */
+    sa_dtype dtype;        /* element type of Q, K, V, O, sink_k, sink_v */
+    float softmax_scale;   /* logit scale; 0 selects 1/sqrt(head_dim) */
+} sa_shape;
+
+/* Number of tiles nt = frames * ceil(tokens / tile); -1 for an invalid shape. */
+int32_t sa_num_tiles(const sa_shape* shape);
+
+/* Length of every kept list for budget k: tpf + min(k, C), C the number of tiles
+ * outside one frame that have at least one key row.  -1 for an invalid shape or k < 0. */
+int32_t sa_max_kept(const sa_shape* shape, int32_t k);
+
+/*
+ * Step 1 - tile pooling (Zebra3D abstract: tiles and their landmark summaries;
+ * AVGGT technical summary 2.B.2: a mean key/value pair stands for discarded columns).
+ *
+ *   q_pool[h][j][:] = mean of q over every row of tile j                 (f32 [bh][nt][d])
+ *   k_pool[h][j][:] = mean of k over the key rows of tile j (0 if none)  (f32 [bh][nt][d])
+ *   v_pool[h][j][:] = mean of v over the key rows (only if v and v_pool are both non-NULL)
+ *   k_cnt[j]        = number of key rows of tile j                       (int32 [nt])
+ *   sink_k[h][s*n_sink + n][:] = k[h][s*N + n][:]  for n < n_sink  ([bh][S*n_sink][d], dtype)
+ *   sink_v likewise from v.
+ * Means accumulate in f32.  sink_k/sink_v may be NULL only when n_sink == 0; sink_v is
+ * required whenever n_sink > 0 and v is non-NULL.
+ */
+sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, const void* v_or_null,
+                       float* q_pool, float* k_pool, float* v_pool_or_null, int32_t* k_cnt,
+                       void* sink_k_or_null, void* sink_v_or_null, sa_stream_t stream);
+
+/*
+ * Step 2 - tile scores (SAF3R abstract: rank the candidate interactions per head).
+ *
+ *   scores[h][i][j] = sum_e q_pool[h][i][e] * k_pool[h][j][e]     (f32 [bh][nt][nt])
+ *
+ * Exact f32 dot products (SIMT FMA, e ascending).  No 1/sqrt(d): it does not change a ranking.
+ */
+sa_status sa_tile_scores(const sa_shape* shape, const float* q_pool, const float* k_pool,
+                         float* scores, sa_stream_t stream);
+
+/* Bytes of workspace sa_select_topk needs: 0 when scores are given (streamed == 0); with
+ * streamed != 0 the size of one L2-resident block of score rows (a few tens of MB at most). */
+size_t sa_select_workspace_size(const sa_shape* shape, int32_t streamed);
+
+/*
+ * Step 3 - top-k tile selection (SAF3R abstract: dynamic, input-dependent selection; AVGGT
+ * technical summary 2.B.1/2.B.2: the own frame and the diagonal are always kept).
+ *
+ * For query tile i of head h in frame f: the kept list is every tile of frame f plus the k
+ * highest-scoring candidate tiles (tiles of other frames with at least one key row), ranked
+ * by score descending and, among equal scores, by lower tile index; all candidates when k
+ * is at least their number.  Output:
+ *   kept_idx[h][i][0..kept_cnt) ascending tile indices, the rest of the row set to -1
+ *                               (int32 [bh][nt][max_kept], max_kept = sa_max_kept(shape,k))
+ *   kept_cnt[h][i]              list length                  (int32 [bh][nt])
+ * scores_or_null != NULL: read the materialised matrix of sa_tile_scores.
+ * scores_or_null == NULL: "streamed" mode - the scores are recomputed from q_pool/k_pool one
+ *   block of rows at a time into `workspace` (>= sa_select_workspace_size(shape, 1) bytes),
+ *   so the [bh][nt][nt] matrix is never materialised.  q_pool/k_pool are ignored otherwise.
+ * Scores that are NaN give unspecified (but in-range) lists.  nt <= 32768 is built.
+ */
+sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null,
+                         const float* q_pool, const float* k_pool, int32_t k,
+                         int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
+                         void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream);
+
+/* Bytes of workspace sa_sparse_attn_fwd needs (0 unless landmark mode on the bf16 path). */
+size_t sa_sparse_attn_workspace_size(const sa_shape* shape, int32_t landmark);
+
+/*
+ * Step 4 - block-sparse attention forward (Zebra3D abstract: tile-sparse attention with
+ * landmark summaries of the unselected context; AVGGT 2.B.2: all queries and special tokens
+ * kept, discarded columns approximated by mean key/value pairs).
+ *
+ * For every query row r of query tile i (head h) the attended keys are
+ *   (i)   the key rows of every tile listed in kept_idx[h][i][0..kept_cnt[h][i]),
+ *   (ii)  every frame's sink token, once each (sink_k/sink_v from sa_tile_pool),
+ *   (iii) if landmark != 0: one token (k_pool[h][j], v_pool[h][j]) with logit bias ln(k_cnt[j])
+ *         for every tile j that is not listed and has k_cnt[j] > 0,
+ * and   O[h][r] = sum_t softmax_t(scale * q_r . k_t + b_t) v_t,
+ *       lse[h][r] = ln sum_t exp(scale * q_r . k_t + b_t)       (natural log; optional).
+ * O has the shape's dtype, [bh][S*N][d]; lse is f32 [bh][S*N].  Products run on the tensor
+ * cores (bf16 in, f32 accumulate; landmark means enter rounded to bf16) with an f32 softmax.
+ * Lists must be ascending with entries in [0, nt) and no repeats; a list from sa_select_topk
+ * always is.  Entries beyond kept_cnt are ignored.  An out-of-range entry is skipped and
+ * reported as SA_ERR_BAD_LIST by sa_check_device_error.
+ * workspace: >= sa_sparse_attn_workspace_size(shape, landmark) bytes (NULL when that is 0).
+ */
+sa_status sa_sparse_attn_fwd(const sa_shape* shape, const void* q, const void* k, const void* v,
+                             const int32_t* kept_idx, const int32_t* kept_cnt, int32_t max_kept,
+                             const void* sink_k_or_null, const void* sink_v_or_null,
+                             int32_t landmark, const float* k_pool_or_null,
+                             const float* v_pool_or_null, const int32_t* k_cnt_or_null,
+                             void* workspace_or_null, size_t workspace_bytes,
+                             void* o, float* lse_or_null, sa_stream_t stream);
+
+/*
+ * The dense control: softmax(scale * Q K^T) V over all S*N keys of each head, no tiles,
+ * sinks or landmarks ("AVGGT" section 1: global attention; "(Full) Attention is More Than
+ * You Need": full attention).  Same layouts and precision as sa_sparse_attn_fwd.
+ */
+sa_status sa_dense_attn_fwd(const sa_shape* shape, const void* q, const void* k, const void* v,
+                            void* o, float* lse_or_null, sa_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char* sa_status_string(sa_status status);
+
+/* Synchronises `stream`, then returns and clears the first device-detected error on the
+ * current device (SA_OK if none).  Returns SA_ERR_CUDA if the synchronisation itself fails. */
+sa_status sa_check_device_error(sa_stream_t stream);
+
+/* Upper bound in nanoseconds on every device-side wait of later launches on the current
+ * device (default 2e9, i.e. 2 s; must be > 0).  A wait that runs out ends its kernel early
+ * with SA_ERR_TIMEOUT recorded; outputs of that launch are then undefined. */
+sa_status sa_set_wait_limit_ns(int64_t limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H_ */

@@ -1,0 +1,96 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every declared symbol, and its
+host-side logic (tile counts, list lengths, argument validation) agrees with the oracle."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import oracle as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from view_recon_b200 import _build, sa
+    _build.build()
+    return sa.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(sa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_and_binding_agree():
+    from view_recon_b200 import sa
+    assert declared_symbols() == sorted(sa.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+@pytest.mark.parametrize("S,N,T,ns,k", [(16, 1374, 128, 5, 35), (4, 256, 64, 0, 4), (3, 7, 2, 2, 1),
+                                        (1, 700, 128, 5, 9), (5, 300, 64, 5, 1000), (2, 4, 2, 2, 5)])
+def test_tile_counts_and_list_lengths(lib, S, N, T, ns, k):
+    from view_recon_b200 import sa
+    g = orc.Geometry(S, N, T, ns)
+    shp = sa.shape(3, S, N, 64, T, ns, "bf16")
+    assert sa.sa_num_tiles(shp) == g.nt
+    assert sa.sa_max_kept(shp, k) == orc.max_kept(g, k)
+
+
+def test_invalid_shapes(lib):
+    from view_recon_b200 import sa
+    assert sa.sa_num_tiles(sa.shape(0, 2, 10)) == -1
+    assert sa.sa_num_tiles(sa.shape(1, 2, 10, n_sink=10)) == -1
+    assert sa.sa_max_kept(sa.shape(1, 2, 10), -1) == -1
+    assert sa.status_string(sa.SA_ERR_TIMEOUT) == "device wait timed out"
+
+
+def test_validation_happens_before_any_launch(lib):
+    # NULL or misaligned pointers are rejected on the host; no CUDA call is made
+    from view_recon_b200 import sa
+    shp = sa.shape(2, 4, 300, 64, 128, 5, "bf16")
+    s = ctypes.byref(shp)
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    odd = P(0x10008)
+    assert lib.sa_tile_pool(s, None, fake, None, fake, fake, None, fake, fake, None, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_tile_pool(s, odd, fake, None, fake, fake, None, fake, fake, None, None) == sa.SA_ERR_INVALID_ARG
+    # sinks present but no sink buffer
+    assert lib.sa_tile_pool(s, fake, fake, None, fake, fake, None, fake, None, None, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_tile_scores(s, fake, None, fake, None) == sa.SA_ERR_INVALID_ARG
+    # max_kept smaller than the list length the budget needs
+    assert lib.sa_select_topk(s, fake, None, None, 3, fake, fake, 2, None, 0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_select_topk(s, fake, None, None, -1, fake, fake, 20, None, 0, None) == sa.SA_ERR_INVALID_ARG
+    # streamed selection without its workspace
+    assert lib.sa_select_topk(s, None, fake, fake, 3, fake, fake, 20, None, 0, None) == sa.SA_ERR_WORKSPACE
+    # landmark mode without pools
+    assert lib.sa_sparse_attn_fwd(s, fake, fake, fake, fake, fake, 6, fake, fake, 1, None, None, None, None, 0,
+                                  fake, None, None) == sa.SA_ERR_INVALID_ARG
+    # head_dim other than 64 is not built
+    bad = sa.shape(2, 4, 300, 32, 128, 0, "bf16")
+    assert lib.sa_dense_attn_fwd(ctypes.byref(bad), fake, fake, fake, fake, None, None) == sa.SA_ERR_UNSUPPORTED
+
+
+def test_workspace_sizes(lib):
+    from view_recon_b200 import sa
+    shp = sa.shape(16, 1024, 1374, 64, 128, 5, "bf16")
+    assert sa.sa_select_workspace_size(shp, False) == 0
+    ws = sa.sa_select_workspace_size(shp, True)
+    assert 0 < ws <= 64 << 20 and ws % (11264 * 4) == 0  # whole score rows, L2-sized
+    shp4 = sa.shape(16, 512, 1374, 64, 128, 5, "bf16")
+    assert sa.sa_sparse_attn_workspace_size(shp4, False) == 0
+    assert sa.sa_sparse_attn_workspace_size(shp4, True) >= 2 * 16 * 5632 * 64 * 2 + 5632 * 4
+
+
+def test_package_fails_loudly_without_library(tmp_path):
+    from view_recon_b200 import sa
+    with pytest.raises(OSError):
+        sa._lib = None
+        sa.load(str(tmp_path / "missing.so"))
+    sa._lib = None

@@ -1,0 +1,519 @@
+// Host side of libsa: argument validation, TMA descriptors and launches for the C-ABI
+// declared in include/sa.h.  All kernels live in the headers included below (one
+// translation unit, so the device error word is shared by every kernel).
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "k_attn_simt.cuh"
+#include "k_attn_tc.cuh"
+#include "k_pool.cuh"
+#include "k_scores.cuh"
+#include "k_select.cuh"
+
+namespace {
+
+constexpr int kTcSlots = 2;
+constexpr int kTcStages = 5;
+constexpr int kMaxDevices = 64;
+
+struct Geo {
+    int64_t bh, S, N, d, T, n_sink, tpf, nt, L;
+    bool bf16;
+    float scale;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sa_status geo_of(const sa_shape* s, Geo* g) {
+    if (!s) return SA_ERR_INVALID_ARG;
+    if (s->bh < 1 || s->frames < 1 || s->tokens < 1 || s->head_dim < 1 || s->tile < 1 || s->n_sink < 0 ||
+        s->n_sink >= s->tokens)
+        return SA_ERR_INVALID_ARG;
+    if (s->dtype != SA_F32 && s->dtype != SA_BF16) return SA_ERR_INVALID_ARG;
+    if (!(s->softmax_scale >= 0.0f) || isinf(s->softmax_scale)) return SA_ERR_INVALID_ARG;
+    g->bh = s->bh;
+    g->S = s->frames;
+    g->N = s->tokens;
+    g->d = s->head_dim;
+    g->T = s->tile;
+    g->n_sink = s->n_sink;
+    g->tpf = (s->tokens + s->tile - 1) / s->tile;
+    g->nt = g->S * g->tpf;
+    g->L = g->S * g->N;
+    g->bf16 = s->dtype == SA_BF16;
+    g->scale = s->softmax_scale > 0.0f ? s->softmax_scale : (float)(1.0 / sqrt((double)s->head_dim));
+    if (g->bh * g->L >= (int64_t(1) << 31) || g->nt >= (int64_t(1) << 31)) return SA_ERR_UNSUPPORTED;
+    if (s->head_dim != 64) return SA_ERR_UNSUPPORTED;
+    if (s->tile != 64 && s->tile != 128) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+int64_t candidate_slots(const Geo& g) {
+    int64_t n = 0;
+    for (int64_t slot = 0; slot < g.tpf; ++slot) {
+        const int64_t n0 = slot * g.T;
+        const int64_t nq = std::min<int64_t>(g.T, g.N - n0);
+        if (nq > std::max<int64_t>(0, g.n_sink - n0)) ++n;
+    }
+    return n;
+}
+
+int64_t max_kept_of(const Geo& g, int64_t k) {
+    const int64_t c = (g.S - 1) * candidate_slots(g);
+    return g.tpf + std::min(k, c);
+}
+
+sa_status launch_status() {
+    const cudaError_t e = cudaPeekAtLastError();
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    return SA_OK;
+}
+
+// ---- per-device one-time kernel attributes
+std::mutex g_attr_mu;
+bool g_attr_done[kMaxDevices];
+
+sa_status ensure_attributes() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    if (g_attr_done[dev]) return SA_OK;
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_simt_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_simt_kernel<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               200 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SEL_MAX_NT * 4) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    g_attr_done[dev] = true;
+    return SA_OK;
+}
+
+// ---- TMA descriptor encoding through the driver entry point (no link-time libcuda)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::mutex g_enc_mu;
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encoder() {
+    std::lock_guard<std::mutex> lk(g_enc_mu);
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        else
+            cudaGetLastError();
+    }
+    return g_encode;
+}
+
+// [rows][64] bf16 matrix, 128-row boxes with the 128-byte swizzle.
+bool encode_rows_bf16(CUtensorMap* m, const void* base, int64_t rows) {
+    EncodeTiledFn enc = encoder();
+    if (!enc || rows < 1) return false;
+    const cuuint64_t dims[2] = {64, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct LandmarkWs {
+    size_t lk, lv, bias, total;
+};
+LandmarkWs landmark_ws(const Geo& g) {
+    const int64_t ntp = (g.nt + 127) / 128 * 128;
+    LandmarkWs w;
+    w.lk = 0;
+    w.lv = align256((size_t)g.bh * ntp * 64 * 2);
+    w.bias = w.lv + align256((size_t)g.bh * ntp * 64 * 2);
+    w.total = w.bias + align256((size_t)ntp * 4);
+    return w;
+}
+
+bool use_tc(const Geo& g) { return g.bf16 && g.T == 128 && g.d == 64; }
+
+size_t select_rows_per_block(const Geo& g) {
+    // one block of score rows stays in L2 (about 48 MB), at least 64 rows
+    int64_t r = (48ll << 20) / (g.nt * 4);
+    r = std::max<int64_t>(64, r / 64 * 64);
+    return (size_t)std::min<int64_t>(r, g.nt);
+}
+
+sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v, const int32_t* kept_idx,
+                      const int32_t* kept_cnt, int32_t max_kept, const void* sink_k, const void* sink_v,
+                      int32_t landmark, const float* k_pool, const float* v_pool, const int32_t* k_cnt,
+                      void* ws, size_t ws_bytes, void* o, float* lse, bool dense, cudaStream_t stream) {
+    sa_status st = ensure_attributes();
+    if (st != SA_OK) return st;
+    if (use_tc(g)) {
+        TcArgs a;
+        memset(&a, 0, sizeof(a));
+        const int64_t ntp = (g.nt + 127) / 128 * 128;
+        const int64_t n_sink_rows = g.S * g.n_sink;
+        bool ok = encode_rows_bf16(&a.tm_q, q, g.bh * g.L) && encode_rows_bf16(&a.tm_k, k, g.bh * g.L) &&
+                  encode_rows_bf16(&a.tm_v, v, g.bh * g.L);
+        if (!dense && n_sink_rows > 0)
+            ok = ok && encode_rows_bf16(&a.tm_sk, sink_k, g.bh * n_sink_rows) &&
+                 encode_rows_bf16(&a.tm_sv, sink_v, g.bh * n_sink_rows);
+        else
+            a.tm_sk = a.tm_k, a.tm_sv = a.tm_v;
+        LandmarkWs lw = landmark_ws(g);
+        if (!dense && landmark) {
+            uint8_t* base = static_cast<uint8_t*>(ws);
+            ok = ok && encode_rows_bf16(&a.tm_lk, base + lw.lk, g.bh * ntp) &&
+                 encode_rows_bf16(&a.tm_lv, base + lw.lv, g.bh * ntp);
+            a.lbias2 = reinterpret_cast<const float*>(base + lw.bias);
+        } else {
+            a.tm_lk = a.tm_k, a.tm_lv = a.tm_v;
+        }
+        if (!ok) return SA_ERR_CUDA;
+        if (!dense && landmark) {
+            uint8_t* base = static_cast<uint8_t*>(ws);
+            const int64_t n4 = g.bh * ntp * 16;
+            const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 148 * 32);
+            landmark_prep_kernel<<<blocks, 256, 0, stream>>>(
+                k_pool, v_pool, k_cnt, reinterpret_cast<__nv_bfloat16*>(base + lw.lk),
+                reinterpret_cast<__nv_bfloat16*>(base + lw.lv), reinterpret_cast<float*>(base + lw.bias),
+                (int32_t)g.bh, (int32_t)g.nt, (int32_t)ntp);
+            if ((st = launch_status()) != SA_OK) return st;
+        }
+        a.kept_idx = kept_idx;
+        a.kept_cnt = kept_cnt;
+        a.o = static_cast<__nv_bfloat16*>(o);
+        a.lse = lse;
+        a.max_kept = max_kept;
+        a.frames = (int32_t)g.S;
+        a.tokens = (int32_t)g.N;
+        a.n_sink = (int32_t)g.n_sink;
+        a.tpf = (int32_t)g.tpf;
+        a.nt = (int32_t)g.nt;
+        a.L = (int32_t)g.L;
+        a.ntp = (int32_t)ntp;
+        a.n_sink_rows = (int32_t)n_sink_rows;
+        a.n_sink_tiles = dense ? 0 : (int32_t)((n_sink_rows + 127) / 128);
+        a.n_lm_chunks = (!dense && landmark) ? (int32_t)(ntp / 128) : 0;
+        a.dense = dense ? 1 : 0;
+        a.landmark = (!dense && landmark) ? 1 : 0;
+        a.q_per_head = dense ? (int32_t)((g.L + 127) / 128) : (int32_t)g.nt;
+        a.total_items = (int32_t)(g.bh * a.q_per_head);
+        a.scale_log2 = (float)((double)g.scale * 1.4426950408889634);
+        using Lay = TcLayout<kTcSlots, kTcStages>;
+        const int mask_words = a.landmark ? (a.nt + 31) / 32 : 0;
+        const size_t smem = Lay::smem_bytes(mask_words);
+        if (smem > 227 * 1024) return SA_ERR_UNSUPPORTED;
+        const int grid = (a.total_items + kTcSlots - 1) / kTcSlots;
+        attn_tc_kernel<kTcSlots, kTcStages><<<grid, Lay::kThreads, smem, stream>>>(a);
+        return launch_status();
+    }
+    AttnArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.max_kept = max_kept;
+    a.sink_k = sink_k;
+    a.sink_v = sink_v;
+    a.landmark = dense ? 0 : landmark;
+    a.k_pool = k_pool;
+    a.v_pool = v_pool;
+    a.k_cnt = k_cnt;
+    a.o = o;
+    a.lse = lse;
+    a.bh = (int32_t)g.bh;
+    a.frames = (int32_t)g.S;
+    a.tokens = (int32_t)g.N;
+    a.tile = (int32_t)g.T;
+    a.n_sink = (int32_t)g.n_sink;
+    a.tpf = (int32_t)g.tpf;
+    a.nt = (int32_t)g.nt;
+    a.L = (int32_t)g.L;
+    a.dense = dense ? 1 : 0;
+    a.scale = g.scale;
+    const int64_t q_per_head = dense ? (g.L + g.T - 1) / g.T : g.nt;
+    const int64_t grid = g.bh * q_per_head;
+    const size_t smem = (size_t)g.T * 64 * 4 * 2 + g.T * 4 + (size_t)((g.nt + 31) / 32) * 4;
+    if (smem > 200 * 1024 || grid >= (int64_t(1) << 31)) return SA_ERR_UNSUPPORTED;
+    if (g.bf16) {
+        if (g.T == 64)
+            attn_simt_kernel<__nv_bfloat16, 64><<<(unsigned)grid, 64, smem, stream>>>(a);
+        else
+            attn_simt_kernel<__nv_bfloat16, 128><<<(unsigned)grid, 128, smem, stream>>>(a);
+    } else {
+        if (g.T == 64)
+            attn_simt_kernel<float, 64><<<(unsigned)grid, 64, smem, stream>>>(a);
+        else
+            attn_simt_kernel<float, 128><<<(unsigned)grid, 128, smem, stream>>>(a);
+    }
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t sa_num_tiles(const sa_shape* shape) {
+    Geo g;
+    if (geo_of(shape, &g) == SA_ERR_INVALID_ARG) return -1;
+    return (int32_t)g.nt;
+}
+
+int32_t sa_max_kept(const sa_shape* shape, int32_t k) {
+    Geo g;
+    if (k < 0 || geo_of(shape, &g) == SA_ERR_INVALID_ARG) return -1;
+    return (int32_t)max_kept_of(g, k);
+}
+
+const char* sa_status_string(sa_status s) {
+    switch (s) {
+        case SA_OK: return "ok";
+        case SA_ERR_INVALID_ARG: return "invalid argument";
+        case SA_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case SA_ERR_CUDA: return "CUDA error";
+        case SA_ERR_TIMEOUT: return "device wait timed out";
+        case SA_ERR_BAD_LIST: return "kept list entry out of range";
+        case SA_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+sa_status sa_check_device_error(sa_stream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    int code = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&code, g_sa_error, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_sa_error, &zero, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    return (sa_status)code;
+}
+
+sa_status sa_set_wait_limit_ns(int64_t limit_ns) {
+    if (limit_ns <= 0) return SA_ERR_INVALID_ARG;
+    const unsigned long long v = (unsigned long long)limit_ns;
+    if (cudaMemcpyToSymbol(g_sa_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    return SA_OK;
+}
+
+sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, const void* v_or_null,
+                       float* q_pool, float* k_pool, float* v_pool_or_null, int32_t* k_cnt, void* sink_k_or_null,
+                       void* sink_v_or_null, sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    if (!q || !k || !q_pool || !k_pool || !k_cnt) return SA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(k_cnt))
+        return SA_ERR_INVALID_ARG;
+    const bool with_v = v_or_null && v_pool_or_null;
+    if ((v_or_null && !aligned16(v_or_null)) || (v_pool_or_null && !aligned16(v_pool_or_null)))
+        return SA_ERR_INVALID_ARG;
+    if (g.n_sink > 0) {
+        if (!sink_k_or_null || !aligned16(sink_k_or_null)) return SA_ERR_INVALID_ARG;
+        if (v_or_null && (!sink_v_or_null || !aligned16(sink_v_or_null))) return SA_ERR_INVALID_ARG;
+    }
+    PoolArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v_or_null;
+    a.q_pool = q_pool;
+    a.k_pool = k_pool;
+    a.v_pool = with_v ? v_pool_or_null : nullptr;
+    a.k_cnt = k_cnt;
+    a.sink_k = g.n_sink > 0 ? sink_k_or_null : nullptr;
+    a.sink_v = (g.n_sink > 0 && v_or_null) ? sink_v_or_null : nullptr;
+    a.bh = (int32_t)g.bh;
+    a.frames = (int32_t)g.S;
+    a.tokens = (int32_t)g.N;
+    a.tile = (int32_t)g.T;
+    a.n_sink = (int32_t)g.n_sink;
+    a.tpf = (int32_t)g.tpf;
+    a.nt = (int32_t)g.nt;
+    const int64_t warps = g.bh * g.nt;
+    const int64_t blocks = (warps + 7) / 8;
+    if (blocks >= (int64_t(1) << 31)) return SA_ERR_UNSUPPORTED;
+    if (g.bf16)
+        pool_tiles_bf16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    else
+        pool_tiles_f32_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    return launch_status();
+}
+
+sa_status sa_tile_scores(const sa_shape* shape, const float* q_pool, const float* k_pool, float* scores,
+                         sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    if (!q_pool || !k_pool || !scores || !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(scores))
+        return SA_ERR_INVALID_ARG;
+    if (g.bh > 65535) return SA_ERR_UNSUPPORTED;
+    ScoreArgs a;
+    a.q_pool = q_pool;
+    a.k_pool = k_pool;
+    a.out = scores;
+    a.ldo = g.nt;
+    a.nt = (int32_t)g.nt;
+    a.h0 = 0;
+    a.i0 = 0;
+    a.rows = (int32_t)g.nt;
+    const dim3 grid((unsigned)((g.nt + 63) / 64), (unsigned)((g.nt + 63) / 64), (unsigned)g.bh);
+    if ((g.nt + 63) / 64 > 65535) return SA_ERR_UNSUPPORTED;
+    tile_scores_kernel<<<grid, 256, 0, stream>>>(a);
+    return launch_status();
+}
+
+size_t sa_select_workspace_size(const sa_shape* shape, int32_t streamed) {
+    Geo g;
+    if (geo_of(shape, &g) != SA_OK) return 0;
+    if (!streamed) return 0;
+    return select_rows_per_block(g) * (size_t)g.nt * 4;
+}
+
+sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, const float* q_pool,
+                         const float* k_pool, int32_t k, int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
+                         void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    if (k < 0 || !kept_idx || !kept_cnt || !aligned16(kept_idx) || !aligned16(kept_cnt)) return SA_ERR_INVALID_ARG;
+    if (max_kept < max_kept_of(g, k)) return SA_ERR_INVALID_ARG;
+    if (g.nt > SEL_MAX_NT) return SA_ERR_UNSUPPORTED;
+    if (scores_or_null) {
+        if (!aligned16(scores_or_null)) return SA_ERR_INVALID_ARG;
+        if (g.bh > 65535) return SA_ERR_UNSUPPORTED;
+    } else {
+        if (!q_pool || !k_pool || !aligned16(q_pool) || !aligned16(k_pool)) return SA_ERR_INVALID_ARG;
+        const size_t need = sa_select_workspace_size(shape, 1);
+        if (!workspace_or_null || workspace_bytes < need || !aligned16(workspace_or_null)) return SA_ERR_WORKSPACE;
+    }
+    if ((st = ensure_attributes()) != SA_OK) return st;
+    SelectArgs a;
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.nt = (int32_t)g.nt;
+    a.tpf = (int32_t)g.tpf;
+    a.tile = (int32_t)g.T;
+    a.tokens = (int32_t)g.N;
+    a.n_sink = (int32_t)g.n_sink;
+    a.k = k;
+    a.max_kept = max_kept;
+    const size_t smem = (size_t)g.nt * 4;
+    if (scores_or_null) {
+        a.scores = scores_or_null;
+        a.lds = g.nt;
+        a.h0 = 0;
+        a.i0 = 0;
+        a.rows = (int32_t)g.nt;
+        select_topk_kernel<<<dim3((unsigned)g.nt, (unsigned)g.bh), SEL_THREADS, smem, stream>>>(a);
+        return launch_status();
+    }
+    // streamed: score one L2-resident block of rows at a time, then select from it
+    const int64_t R = (int64_t)select_rows_per_block(g);
+    float* blk = static_cast<float*>(workspace_or_null);
+    for (int64_t h = 0; h < g.bh; ++h) {
+        for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
+            const int64_t rows = std::min<int64_t>(R, g.nt - i0);
+            ScoreArgs sc;
+            sc.q_pool = q_pool;
+            sc.k_pool = k_pool;
+            sc.out = blk;
+            sc.ldo = g.nt;
+            sc.nt = (int32_t)g.nt;
+            sc.h0 = (int32_t)h;
+            sc.i0 = (int32_t)i0;
+            sc.rows = (int32_t)rows;
+            tile_scores_kernel<<<dim3((unsigned)((g.nt + 63) / 64), (unsigned)((rows + 63) / 64), 1), 256, 0,
+                                 stream>>>(sc);
+            if ((st = launch_status()) != SA_OK) return st;
+            a.scores = blk;
+            a.lds = g.nt;
+            a.h0 = (int32_t)h;
+            a.i0 = (int32_t)i0;
+            a.rows = (int32_t)rows;
+            select_topk_kernel<<<dim3((unsigned)rows, 1), SEL_THREADS, smem, stream>>>(a);
+            if ((st = launch_status()) != SA_OK) return st;
+        }
+    }
+    return SA_OK;
+}
+
+size_t sa_sparse_attn_workspace_size(const sa_shape* shape, int32_t landmark) {
+    Geo g;
+    if (geo_of(shape, &g) != SA_OK) return 0;
+    if (!landmark || !use_tc(g)) return 0;
+    return landmark_ws(g).total;
+}
+
+sa_status sa_sparse_attn_fwd(const sa_shape* shape, const void* q, const void* k, const void* v,
+                             const int32_t* kept_idx, const int32_t* kept_cnt, int32_t max_kept,
+                             const void* sink_k_or_null, const void* sink_v_or_null, int32_t landmark,
+                             const float* k_pool_or_null, const float* v_pool_or_null,
+                             const int32_t* k_cnt_or_null, void* workspace_or_null, size_t workspace_bytes,
+                             void* o, float* lse_or_null, sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    if (!q || !k || !v || !kept_idx || !kept_cnt || !o) return SA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(kept_idx) || !aligned16(kept_cnt) ||
+        !aligned16(o) || (lse_or_null && !aligned16(lse_or_null)))
+        return SA_ERR_INVALID_ARG;
+    if (max_kept < 1 || max_kept > g.nt) return SA_ERR_INVALID_ARG;
+    if (g.n_sink > 0 && (!sink_k_or_null || !sink_v_or_null || !aligned16(sink_k_or_null) ||
+                         !aligned16(sink_v_or_null)))
+        return SA_ERR_INVALID_ARG;
+    if (landmark) {
+        if (!k_pool_or_null || !v_pool_or_null || !k_cnt_or_null || !aligned16(k_pool_or_null) ||
+            !aligned16(v_pool_or_null) || !aligned16(k_cnt_or_null))
+            return SA_ERR_INVALID_ARG;
+        if (g.nt > 16384) return SA_ERR_UNSUPPORTED;
+        const size_t need = sa_sparse_attn_workspace_size(shape, 1);
+        if (need && (!workspace_or_null || workspace_bytes < need || !aligned16(workspace_or_null)))
+            return SA_ERR_WORKSPACE;
+    }
+    return attn_common(g, q, k, v, kept_idx, kept_cnt, max_kept, sink_k_or_null, sink_v_or_null, landmark ? 1 : 0,
+                       k_pool_or_null, v_pool_or_null, k_cnt_or_null, workspace_or_null, workspace_bytes, o,
+                       lse_or_null, false, stream);
+}
+
+sa_status sa_dense_attn_fwd(const sa_shape* shape, const void* q, const void* k, const void* v, void* o,
+                            float* lse_or_null, sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    if (!q || !k || !v || !o) return SA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse_or_null && !aligned16(lse_or_null)))
+        return SA_ERR_INVALID_ARG;
+    return attn_common(g, q, k, v, nullptr, nullptr, 0, nullptr, nullptr, 0, nullptr, nullptr, nullptr, nullptr, 0,
+                       o, lse_or_null, true, stream);
+}
+
+}  // extern "C"
