@@ -109,6 +109,19 @@ class SparseGlobalAttention:
 
     __call__ = forward
 
+    def launches_per_call(self) -> int:
+        """Kernel launches libsa makes for one forward (for launch accounting)."""
+        n = 1  # pooling
+        if self.streamed:
+            rows = sa.sa_select_workspace_size(self.shape, True) // (4 * self.nt)
+            n += 2 * self.bh * (-(-self.nt // rows))  # score block + select block
+        else:
+            n += 2  # scores + select
+        n += 1  # attention
+        if self.landmark and sa.sa_sparse_attn_workspace_size(self.shape, True) > 0:
+            n += 1  # landmark tables
+        return n
+
 
 def dense_attention(q, k, v, frames: int, tokens: int, dtype: str = "bf16", with_lse: bool = True, stream=None):
     """Dense control on device tensors [bh][S*N][64]; returns (O, LSE)."""
