@@ -246,7 +246,7 @@ def run_ours(args, w):
 
     import synth
     from view_recon_b200 import sa
-    from view_recon_b200.pipeline import SparseGlobalAttention, dense_attention
+    from view_recon_b200.pipeline import SparseGlobalAttention
 
     rank, world, local = rank_env()
     if world > 1:
@@ -316,18 +316,17 @@ def run_ours(args, w):
     ms_pool, ms_score, ms_select, ms_attn = (float(x) for x in stage.mean(axis=0))
 
     # dense control at the same shape (speedup reference)
-    od = torch.empty_like(q)
-    ld = torch.empty((w.heads, w.L), dtype=torch.float32, device=dev)
-    shp_d = sa.shape(w.heads, w.frames, w.tokens, w.head_dim, w.tile, 0, w.dtype)
+    from view_recon_b200.pipeline import DenseAttention
+    dense = DenseAttention(w.heads, w.frames, w.tokens, w.dtype, w.head_dim, device=dev)
     n_dense = max(3, min(10, args.steps))
     for _ in range(2):
-        sa.sa_dense_attn_fwd(shp_d, q, k, v, od, ld)
+        dense(q, k, v)
     d_ms = []
     for _ in range(n_dense):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        sa.sa_dense_attn_fwd(shp_d, q, k, v, od, ld)
+        dense(q, k, v)
         e1.record(stream)
         d_ms.append((e0, e1))
     torch.cuda.synchronize(dev)

@@ -146,7 +146,9 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null,
                          int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
                          void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream);
 
-/* Bytes of workspace sa_sparse_attn_fwd needs (0 unless landmark mode on the bf16 path). */
+/* Bytes of workspace sa_sparse_attn_fwd needs: on the tensor-core path (bf16, tile 128) a
+ * transposed copy of every V tile it may gather (the size of V plus the sink segment) and, in
+ * landmark mode, the bf16 landmark tables; 0 on the CUDA-core path (f32 or tile 64). */
 size_t sa_sparse_attn_workspace_size(const sa_shape* shape, int32_t landmark);
 
 /*
@@ -176,12 +178,18 @@ sa_status sa_sparse_attn_fwd(const sa_shape* shape, const void* q, const void* k
                              void* workspace_or_null, size_t workspace_bytes,
                              void* o, float* lse_or_null, sa_stream_t stream);
 
+/* Bytes of workspace sa_dense_attn_fwd needs (a transposed copy of V on the tensor-core
+ * path, 0 on the CUDA-core path). */
+size_t sa_dense_attn_workspace_size(const sa_shape* shape);
+
 /*
  * The dense control: softmax(scale * Q K^T) V over all S*N keys of each head, no tiles,
  * sinks or landmarks ("AVGGT" section 1: global attention; "(Full) Attention is More Than
- * You Need": full attention).  Same layouts and precision as sa_sparse_attn_fwd.
+ * You Need": full attention).  Same layouts and precision as sa_sparse_attn_fwd; n_sink is
+ * ignored.  workspace: >= sa_dense_attn_workspace_size(shape) bytes (NULL when that is 0).
  */
 sa_status sa_dense_attn_fwd(const sa_shape* shape, const void* q, const void* k, const void* v,
+                            void* workspace_or_null, size_t workspace_bytes,
                             void* o, float* lse_or_null, sa_stream_t stream);
 
 /* Static description of a status code (never NULL). */

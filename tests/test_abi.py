@@ -74,7 +74,12 @@ def test_validation_happens_before_any_launch(lib):
                                   fake, None, None) == sa.SA_ERR_INVALID_ARG
     # head_dim other than 64 is not built
     bad = sa.shape(2, 4, 300, 32, 128, 0, "bf16")
-    assert lib.sa_dense_attn_fwd(ctypes.byref(bad), fake, fake, fake, fake, None, None) == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_dense_attn_fwd(ctypes.byref(bad), fake, fake, fake, None, 0, fake, None, None) == sa.SA_ERR_UNSUPPORTED
+    # the tensor-core path needs its workspace (transposed V tiles)
+    good = sa.shape(2, 4, 300, 64, 128, 0, "bf16")
+    assert lib.sa_dense_attn_fwd(ctypes.byref(good), fake, fake, fake, None, 0, fake, None, None) == sa.SA_ERR_WORKSPACE
+    assert lib.sa_sparse_attn_fwd(s, fake, fake, fake, fake, fake, 6, fake, fake, 0, None, None, None, None, 0,
+                                  fake, None, None) == sa.SA_ERR_WORKSPACE
 
 
 def test_workspace_sizes(lib):
@@ -84,8 +89,14 @@ def test_workspace_sizes(lib):
     ws = sa.sa_select_workspace_size(shp, True)
     assert 0 < ws <= 64 << 20 and ws % (11264 * 4) == 0  # whole score rows, L2-sized
     shp4 = sa.shape(16, 512, 1374, 64, 128, 5, "bf16")
-    assert sa.sa_sparse_attn_workspace_size(shp4, False) == 0
-    assert sa.sa_sparse_attn_workspace_size(shp4, True) >= 2 * 16 * 5632 * 64 * 2 + 5632 * 4
+    vt = 16 * 5632 * 64 * 128 * 2                 # transposed V tiles of every key tile
+    sinks = 16 * 20 * 64 * 128 * 2                # 512 frames x 5 sinks = 2560 rows = 20 tiles
+    assert sa.sa_sparse_attn_workspace_size(shp4, False) == vt + sinks
+    assert sa.sa_sparse_attn_workspace_size(shp4, True) >= vt + sinks + 2 * 16 * 5632 * 64 * 2 + 5632 * 4
+    assert sa.sa_dense_attn_workspace_size(shp4) == 16 * (-(-512 * 1374 // 128)) * 64 * 128 * 2
+    # the CUDA-core path (f32, or tile 64) needs none
+    assert sa.sa_sparse_attn_workspace_size(sa.shape(2, 4, 256, 64, 64, 0, "f32"), True) == 0
+    assert sa.sa_dense_attn_workspace_size(sa.shape(2, 4, 256, 64, 64, 0, "bf16")) == 0
 
 
 def test_package_fails_loudly_without_library(tmp_path):

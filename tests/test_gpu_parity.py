@@ -156,7 +156,7 @@ def test_argument_errors_touch_nothing():
     assert e.value.status == sa.SA_ERR_INVALID_ARG
     bad = sa.shape(w.heads, w.frames, w.tokens, 32, 128, 0, "bf16")
     with pytest.raises(sa.SaError) as e:
-        sa.sa_dense_attn_fwd(bad, q, k, v, layer.buf.o)
+        sa.sa_dense_attn_fwd(bad, q, k, v, None, layer.buf.o)
     assert e.value.status == sa.SA_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert torch.equal(before, layer.buf.o)

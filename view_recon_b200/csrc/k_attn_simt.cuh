@@ -210,33 +210,3 @@ __global__ void __launch_bounds__(TILE) attn_simt_kernel(AttnArgs a) {
         if (a.lse) a.lse[(int64_t)h * a.L + qrow0 + tid] = st.l > 0.0f ? st.m + logf(st.l) : -INFINITY;
     }
 }
-
-// Landmark tables for the tensor-core kernel: bf16 copies of the tile means (zero rows past
-// nt) and the per-tile logit bias log2(c_j) in base-2 units (-inf where c_j = 0 or j >= nt).
-__global__ void landmark_prep_kernel(const float* k_pool, const float* v_pool, const int32_t* k_cnt,
-                                     __nv_bfloat16* lk, __nv_bfloat16* lv, float* lbias2, int32_t bh,
-                                     int32_t nt, int32_t ntp) {
-    const int64_t n4 = (int64_t)bh * ntp * 16;  // float4 groups
-    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n4;
-         idx += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t rowp = idx >> 4;  // h * ntp + j
-        const int c4 = (int)(idx & 15);
-        const int64_t h = rowp / ntp, j = rowp % ntp;
-        float4 x = make_float4(0, 0, 0, 0), y = x;
-        if (j < nt) {
-            x = __ldg(reinterpret_cast<const float4*>(k_pool + (h * nt + j) * 64) + c4);
-            y = __ldg(reinterpret_cast<const float4*>(v_pool + (h * nt + j) * 64) + c4);
-        }
-        uint2 px, py;
-        px.x = pack_bf16x2(x.x, x.y);
-        px.y = pack_bf16x2(x.z, x.w);
-        py.x = pack_bf16x2(y.x, y.y);
-        py.y = pack_bf16x2(y.z, y.w);
-        reinterpret_cast<uint2*>(lk)[idx] = px;
-        reinterpret_cast<uint2*>(lv)[idx] = py;
-        if (h == 0 && c4 == 0) {
-            const int c = j < nt ? k_cnt[j] : 0;
-            lbias2[j] = c > 0 ? log2f((float)c) : -INFINITY;
-        }
-    }
-}

@@ -2,21 +2,28 @@
 // bf16, d = 64, tile = 128 ("Zebra3D" abstract: tile-sparse attention with landmark
 // summaries; "AVGGT" 2.B.2: special tokens kept, discarded columns as mean K/V pairs).
 //
-// One CTA owns NSLOT query tiles ("slots"); each slot walks its own item list:
+// One CTA owns NSLOT = 2 query tiles ("slots"); each slot walks its own item list:
 //   sparse: the listed key tiles, then the sink segment in 128-row chunks, then (landmark
 //           mode) every 128-tile chunk of the landmark table with listed tiles masked out;
 //   dense:  every 128-row key tile of the head.
-// Warp roles (NSLOT = 2 -> 320 threads, one CTA per SM):
-//   warp 0      TMA producer: Q tiles, then the K/V tile of each item into a STAGES-deep
-//               shared-memory ring (128-byte swizzle, gathered by tile index);
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer:
-//                 S_x = Q_x K^T      (M=128, N=128, K=64; both operands K-major in smem)
-//                 O_x += P_x V       (M=128, N=64,  K=128; P from TMEM, V MN-major in smem);
-//   warps 2..   one 128-thread softmax group per slot; thread r owns row r of its slot:
-//               tcgen05.ld of S, masking, base-2 online softmax with a lazy max (the
-//               accumulator is rescaled only when the row max grows by more than 2^8),
-//               P written back to TMEM as bf16, O rescale in TMEM, final normalisation.
-// TMEM columns per slot: S 128 (f32), P 64 (bf16 pairs), O 64 (f32).
+// An item is a K tile ([128 keys][64] bf16, gathered by TMA straight from K) and the
+// matching transposed V tile ([64][128 keys], prepared in the workspace, see
+// k_attn_prep.cuh) so that both products read K-major shared-memory operands.
+// The two slots are fully decoupled, so that one slot's exponentials fill the other's
+// waits (TMEM round trips, barrier hand-offs) instead of running in lockstep with them:
+// each has its own producer warp, its own MMA-issuing warp and its own STAGES-deep ring.
+// Warp roles (384 threads, one CTA per SM):
+//   warps 0, 2      TMA producers of slots 0, 1: the Q tile, then K + V^T of every item
+//                   (128-byte swizzle);
+//   warps 1, 3      tcgen05.mma issuers of slots 0, 1 (one elected lane; warp 1 also owns
+//                   the TMEM allocation):
+//                     S_x = Q_x K^T   (M=128, N=128, K=64; A and B K-major in shared memory)
+//                     O_x += P_x V    (M=128, N=64, K=128; P read from TMEM, V^T K-major);
+//   warpgroup 1+x   the softmax group of slot x; thread r owns row r: tcgen05.ld of its 128
+//                   scores, masking, base-2 online softmax with a lazy max (O is rescaled
+//                   only when the row max grows by more than 2^8), P written back to TMEM
+//                   as bf16, O rescale in TMEM, final normalisation.
+// TMEM columns per slot: S 128 (f32), P 64 (bf16 pairs), O 64 (f32): 512 in total.
 // Every wait is bounded (g_sa_wait_limit_ns): a wait that runs out records SA_ERR_TIMEOUT,
 // raises the CTA abort flag, every role drains what it has in flight and the CTA exits.
 // No TMA multicast and no clusters are used.
@@ -24,33 +31,43 @@
 #include "sa_device.cuh"
 
 struct __align__(64) TcArgs {
-    CUtensorMap tm_q, tm_k, tm_v;    // [bh*L][64] bf16, box 64 x 128
-    CUtensorMap tm_sk, tm_sv;        // [bh*S*n_sink][64] sink segment
-    CUtensorMap tm_lk, tm_lv;        // [bh*ntp][64] landmark tables
+    CUtensorMap tm_q, tm_k;     // [bh*L][64] bf16, box 64 x 128
+    CUtensorMap tm_vt;          // [bh*n_vtiles*64][128] bf16 transposed V tiles, box 64 x 64
+    CUtensorMap tm_sk, tm_svt;  // sink keys [bh*S*n_sink][64]; transposed sink V tiles
+    CUtensorMap tm_lk, tm_lvt;  // landmark keys [bh*ntp][64]; transposed landmark V tiles
     const int32_t* kept_idx;
     const int32_t* kept_cnt;
-    const float* lbias2;             // [ntp] log2(c_j) or -inf
+    const float* lbias2;  // [ntp] log2(c_j) or -inf
     __nv_bfloat16* o;
     float* lse;
     int32_t max_kept;
     int32_t frames, tokens, n_sink, tpf, nt, L, ntp;
+    int32_t n_vtiles;  // transposed V tiles per head (nt, or ceil(L/128) dense)
     int32_t n_sink_rows, n_sink_tiles, n_lm_chunks;
     int32_t dense, landmark;
     int32_t q_per_head, total_items;
+    uint32_t tpf_magic;  // j / tpf == __umulhi(j, tpf_magic) for every tile index j < nt
     float scale_log2;
 };
+
+// Of every 8 column pairs of a score row, this many take their exponentials on the FMA pipe
+// (exp2_poly2) and the rest on the MUFU (ex2.approx).
+#ifndef SA_EXP2_FMA_PAIRS_PER8
+#define SA_EXP2_FMA_PAIRS_PER8 2
+#endif
 
 namespace tc {
 
 constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 64, 1);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 64, 0);  // V^T: K-major B
 
 struct Item {
-    int kind;     // 0 = key tile, 1 = sink chunk, 2 = landmark chunk, -1 = skipped
-    int32_t row;  // first row in the item's tensor map
-    int lo, hi;   // valid key columns [lo, hi)
-    int chunk;    // landmark chunk index
+    int kind;      // 0 = key tile, 1 = sink chunk, 2 = landmark chunk, -1 = skipped
+    int32_t krow;  // first row of the K tile in its tensor map
+    int32_t vrow;  // first row of the V^T tile in its tensor map
+    int lo, hi;    // valid key columns [lo, hi)
+    int chunk;     // landmark chunk index
 };
 
 struct Slot {
@@ -88,29 +105,39 @@ __device__ __forceinline__ Slot make_slot(const TcArgs& a, int item) {
     return s;
 }
 
+__device__ __forceinline__ Item get_item_j(const TcArgs& a, const Slot& s, int n, int j);
+
 __device__ __forceinline__ Item get_item(const TcArgs& a, const Slot& s, int n) {
+    const int j = (!a.dense && n < s.cnt) ? __ldg(s.list + n) : 0;
+    return get_item_j(a, s, n, j);
+}
+
+// Same as get_item with the list entry s.list[n] (when n < s.cnt) supplied by the caller.
+__device__ __forceinline__ Item get_item_j(const TcArgs& a, const Slot& s, int n, int j) {
     Item it;
     it.chunk = 0;
     if (a.dense) {
         it.kind = 0;
-        it.row = s.h * a.L + n * 128;
+        it.krow = s.h * a.L + n * 128;
+        it.vrow = (s.h * a.n_vtiles + n) * 64;
         it.lo = 0;
         it.hi = min(128, a.L - n * 128);
         return it;
     }
     if (n < s.cnt) {
-        const int j = __ldg(s.list + n);
         if (j < 0 || j >= a.nt) {
             it.kind = -1;
-            it.row = s.h * a.L;
+            it.krow = s.h * a.L;
+            it.vrow = s.h * a.n_vtiles * 64;
             it.lo = it.hi = 0;
             return it;
         }
-        const int f = j / a.tpf, slot = j % a.tpf;
+        const int f = (int)__umulhi((uint32_t)j, a.tpf_magic), slot = j - f * a.tpf;
         const int n0 = slot * 128;
         const int nk = min(128, a.tokens - n0);
         it.kind = 0;
-        it.row = s.h * a.L + f * a.tokens + n0;
+        it.krow = s.h * a.L + f * a.tokens + n0;
+        it.vrow = (s.h * a.n_vtiles + j) * 64;
         it.lo = min(nk, max(0, a.n_sink - n0));
         it.hi = nk;
         return it;
@@ -118,14 +145,16 @@ __device__ __forceinline__ Item get_item(const TcArgs& a, const Slot& s, int n) 
     n -= s.cnt;
     if (n < a.n_sink_tiles) {
         it.kind = 1;
-        it.row = s.h * a.n_sink_rows + n * 128;
+        it.krow = s.h * a.n_sink_rows + n * 128;
+        it.vrow = (s.h * a.n_sink_tiles + n) * 64;
         it.lo = 0;
         it.hi = min(128, a.n_sink_rows - n * 128);
         return it;
     }
     n -= a.n_sink_tiles;
     it.kind = 2;
-    it.row = s.h * a.ntp + n * 128;
+    it.krow = s.h * a.ntp + n * 128;
+    it.vrow = (s.h * a.n_lm_chunks + n) * 64;
     it.lo = 0;
     it.hi = 128;
     it.chunk = n;
@@ -144,190 +173,223 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// Warp-uniform bounded wait for a ping-pong token phase, which also ends as soon as the other
+// slot has finished its items (it then no longer passes the token).
+__device__ __forceinline__ bool wait_token(uint64_t* bar, uint32_t parity, volatile int* other_done,
+                                           volatile int* abort_flag) {
+    bool ok = true;
+    if (!mbar_test(bar, parity)) {
+        const uint64_t t0 = sa_globaltimer();
+        const uint64_t limit = g_sa_wait_limit_ns;
+        for (uint32_t it = 1;; ++it) {
+            if (mbar_test(bar, parity) || *other_done) break;
+            if ((it & 63u) == 0) {
+                if (*abort_flag) { ok = false; break; }
+                if (sa_globaltimer() - t0 > limit) {
+                    sa_flag_error(SA_ERR_TIMEOUT);
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+            }
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 }  // namespace tc
 
 template <int NSLOT, int STAGES>
 struct TcLayout {
-    static constexpr int kThreads = 64 + 128 * NSLOT;
-    static constexpr uint32_t kTmemCols = NSLOT == 1 ? 256 : 512;
+    static constexpr int kThreads = 128 + 128 * NSLOT;
+    static constexpr uint32_t kTmemCols = 512;
+    // registers per thread after the split: warpgroup 0 gives, the softmax groups take
+    static constexpr uint32_t kRegsControl = 56;
+    static constexpr uint32_t kRegsSoftmax = 224;
+    static constexpr uint32_t kRegsNeeded = 128 * kRegsControl + 128 * NSLOT * kRegsSoftmax;
     static constexpr int kQ = 0;
-    static constexpr int kKV = NSLOT * tc::kTileBytes;
-    static constexpr int kBars = kKV + STAGES * 2 * tc::kTileBytes;
-    // q_full[N], kv_full[S], kv_empty[S], s_full[N], s_free[N], p_full[N], pv_done[N], drain[1]
-    static constexpr int kNumBars = 5 * NSLOT + 2 * STAGES + 1;
-    static constexpr int kMisc = kBars + 8 * kNumBars;  // tmem base (4 B), abort flag (4 B)
-    static constexpr int kMask = (kMisc + 8 + 15) & ~15;
+    static constexpr int kKV = NSLOT * tc::kTileBytes;                 // [slot][stage] K + V^T
+    static constexpr int kBars = kKV + NSLOT * STAGES * 2 * tc::kTileBytes;
+    // per slot: q_full, kv_full[S], kv_empty[S], s_full, s_free, p_full, pv_done, drain
+    static constexpr int kBarsPerSlot = 6 + 2 * STAGES;
+    // ping-pong tokens: tok[x] completes when the other slot has finished a batch of exponentials
+    static constexpr int kTok = kBars + 8 * kBarsPerSlot * NSLOT;
+    static constexpr int kMisc = kTok + 8 * NSLOT;  // tmem base, abort flag, done[NSLOT]
+    static constexpr int kEnd = kMisc + 16 + 4 * NSLOT;
     static constexpr uint32_t colS(int x) { return x * 128; }
     static constexpr uint32_t colP(int x) { return NSLOT * 128 + x * 64; }
     static constexpr uint32_t colO(int x) { return NSLOT * 128 + NSLOT * 64 + x * 64; }
-    static size_t smem_bytes(int mask_words) { return 1024 + kMask + (size_t)NSLOT * mask_words * 4; }
+    static size_t smem_bytes() { return 1024 + kEnd; }
 };
 
 template <int NSLOT, int STAGES>
-__global__ void __launch_bounds__(64 + 128 * NSLOT, 1) attn_tc_kernel(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __grid_constant__ TcArgs a) {
     using Lay = TcLayout<NSLOT, STAGES>;
+    static_assert(NSLOT == 2, "warp roles are laid out for two slots");
+    static_assert(NSLOT * (128 + 64 + 64) <= 512, "TMEM columns");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = smem + Lay::kQ;
-    uint8_t* sKV = smem + Lay::kKV;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBars);
-    uint64_t* q_full = bars;
-    uint64_t* kv_full = q_full + NSLOT;
-    uint64_t* kv_empty = kv_full + STAGES;
-    uint64_t* s_full = kv_empty + STAGES;
-    uint64_t* s_free = s_full + NSLOT;
-    uint64_t* p_full = s_free + NSLOT;
-    uint64_t* pv_done = p_full + NSLOT;
-    uint64_t* drain_bar = pv_done + NSLOT;
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
-    uint32_t* lmask = reinterpret_cast<uint32_t*>(smem + Lay::kMask);
-    const int mask_words = a.landmark ? (a.nt + 31) / 32 : 0;
+    uint64_t* tok = reinterpret_cast<uint64_t*>(smem + Lay::kTok);             // [NSLOT]
+    volatile int* slot_done = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 16);  // [NSLOT]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    tc::Slot slots[NSLOT];
-#pragma unroll
-    for (int x = 0; x < NSLOT; ++x) slots[x] = tc::make_slot(a, blockIdx.x * NSLOT + x);
-    int max_items = 0;
-#pragma unroll
-    for (int x = 0; x < NSLOT; ++x) max_items = max(max_items, slots[x].n_items);
+    const bool is_softmax = warp >= 4;
+    // the slot this warp works for: control warps 0,1 -> slot 0, 2,3 -> slot 1
+    const int x = is_softmax ? (warp - 4) >> 2 : (warp >> 1);
+    uint8_t* sQ = smem + Lay::kQ + x * tc::kTileBytes;
+    uint8_t* sKV = smem + Lay::kKV + x * STAGES * 2 * tc::kTileBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBars) + x * Lay::kBarsPerSlot;
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = kv_full + STAGES;
+    uint64_t* s_full = kv_empty + STAGES;
+    uint64_t* s_free = s_full + 1;
+    uint64_t* p_full = s_free + 1;
+    uint64_t* pv_done = p_full + 1;
+    uint64_t* drain_bar = pv_done + 1;
 
     if (threadIdx.x == 0) {
-        for (int x = 0; x < NSLOT; ++x) {
-            mbar_init(&q_full[x], 1);
-            mbar_init(&s_full[x], 1);
-            mbar_init(&s_free[x], 128);
-            mbar_init(&p_full[x], 128);
-            mbar_init(&pv_done[x], 1);
+        uint64_t* all = reinterpret_cast<uint64_t*>(smem + Lay::kBars);
+        for (int y = 0; y < NSLOT; ++y) {
+            uint64_t* b = all + y * Lay::kBarsPerSlot;
+            mbar_init(&b[0], 1);  // q_full
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&b[1 + s], 1);           // kv_full
+                mbar_init(&b[1 + STAGES + s], 1);  // kv_empty
+            }
+            mbar_init(&b[1 + 2 * STAGES], 1);      // s_full
+            mbar_init(&b[2 + 2 * STAGES], 128);    // s_free
+            mbar_init(&b[3 + 2 * STAGES], 128);    // p_full
+            mbar_init(&b[4 + 2 * STAGES], 1);      // pv_done
+            mbar_init(&b[5 + 2 * STAGES], 1);      // drain
+            mbar_init(&tok[y], 128);
+            slot_done[y] = 0;
         }
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
-        }
-        mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0 && lane == 0) {
+    if ((warp == 0 || warp == 2) && lane == 0) {
         tma_prefetch_desc(&a.tm_q);
         tma_prefetch_desc(&a.tm_k);
-        tma_prefetch_desc(&a.tm_v);
+        tma_prefetch_desc(&a.tm_vt);
     }
     if (warp == 1) {
         tmem_alloc(tmem_base_smem, Lay::kTmemCols);
         tmem_relinquish();
     }
-    // kept-tile bit masks for the landmark chunks
-    const int sx = warp >= 2 ? (warp - 2) >> 2 : 0;
-    const int st = threadIdx.x - 64 - 128 * sx;  // 0..127 inside a softmax group
-    if (warp >= 2 && mask_words)
-        for (int w = st; w < mask_words; w += 128) lmask[sx * mask_words + w] = 0u;
-    __syncthreads();
-    if (warp >= 2 && mask_words)
-        for (int n = st; n < slots[sx].cnt; n += 128) {
-            const int j = __ldg(slots[sx].list + n);
-            if (j >= 0 && j < a.nt) atomicOr(&lmask[sx * mask_words + (j >> 5)], 1u << (j & 31));
-        }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_smem;
+    const tc::Slot sl = tc::make_slot(a, blockIdx.x * NSLOT + x);
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            uint32_t issued_phase[STAGES];
-            bool issued[STAGES];
-#pragma unroll
-            for (int s = 0; s < STAGES; ++s) issued[s] = false;
+    if (!is_softmax) {
+        setmaxnreg_dec<Lay::kRegsControl>();
+        const int n_items = sl.n_items;
+        if ((warp & 1) == 0) {
+            // -------------------------------------------------------------- TMA producer (slot x)
+            // The whole warp walks the loop (waits are per lane); one elected lane issues.
+            const bool leader = tc::elect_one();
+            uint32_t issued_mask = 0, phase_mask = 0;  // per ring stage: a load was issued / its parity
             bool ok = true;
-            for (int x = 0; x < NSLOT; ++x)
-                if (slots[x].active) {
-                    mbar_arrive_expect_tx(&q_full[x], tc::kTileBytes);
-                    tma_load_2d(sQ + x * tc::kTileBytes, &a.tm_q, &q_full[x], 0, slots[x].qrow);
+            if (n_items > 0 && leader) {
+                mbar_arrive_expect_tx(q_full, tc::kTileBytes);
+                tma_load_2d(sQ, &a.tm_q, q_full, 0, sl.qrow);
+            }
+            for (int n = 0; n < n_items; ++n) {
+                const uint32_t s = n % STAGES, ph = (n / STAGES) & 1u;
+                if (!mbar_wait_warp(&kv_empty[s], ph ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
                 }
-            uint32_t seq = 0;
-            for (int n = 0; n < max_items && ok; ++n) {
-                for (int x = 0; x < NSLOT; ++x) {
-                    if (n >= slots[x].n_items) continue;
-                    const uint32_t s = seq % STAGES, ph = (seq / STAGES) & 1u;
-                    ++seq;
-                    if (!mbar_wait(&kv_empty[s], ph ^ 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const tc::Item it = tc::get_item(a, slots[x], n);
+                if (leader) {
+                    const tc::Item it = tc::get_item(a, sl, n);
                     const CUtensorMap* mk = it.kind == 1 ? &a.tm_sk : (it.kind == 2 ? &a.tm_lk : &a.tm_k);
-                    const CUtensorMap* mv = it.kind == 1 ? &a.tm_sv : (it.kind == 2 ? &a.tm_lv : &a.tm_v);
+                    const CUtensorMap* mv = it.kind == 1 ? &a.tm_svt : (it.kind == 2 ? &a.tm_lvt : &a.tm_vt);
                     uint8_t* dk = sKV + s * 2 * tc::kTileBytes;
                     mbar_arrive_expect_tx(&kv_full[s], 2 * tc::kTileBytes);
-                    tma_load_2d(dk, mk, &kv_full[s], 0, it.row);
-                    tma_load_2d(dk + tc::kTileBytes, mv, &kv_full[s], 0, it.row);
-                    issued[s] = true;
-                    issued_phase[s] = ph;
+                    tma_load_2d(dk, mk, &kv_full[s], 0, it.krow);
+                    tma_load_2d(dk + tc::kTileBytes, mv, &kv_full[s], 0, it.vrow);
+                    tma_load_2d(dk + tc::kTileBytes + tc::kTileBytes / 2, mv, &kv_full[s], 64, it.vrow);
                 }
+                issued_mask |= 1u << s;
+                phase_mask = (phase_mask & ~(1u << s)) | (ph << s);
             }
-            if (!ok) {  // let every copy this thread started land before the CTA exits
+            if (!ok) {  // let every copy this warp started land before the CTA exits
                 for (int s = 0; s < STAGES; ++s)
-                    if (issued[s]) tc::drain_wait(&kv_full[s], issued_phase[s]);
-                for (int x = 0; x < NSLOT; ++x)
-                    if (slots[x].active) tc::drain_wait(&q_full[x], 0);
+                    if ((issued_mask >> s) & 1u) tc::drain_wait(&kv_full[s], (phase_mask >> s) & 1u);
+                if (n_items > 0) tc::drain_wait(q_full, 0);
             }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            bool ok = true;
+        } else {
+            // -------------------------------------------------------------- MMA issuer (slot x)
+            const bool leader = tc::elect_one();
+            bool ok = n_items == 0 || mbar_wait_warp(q_full, 0, abort_flag);
             bool any_mma = false;
-            for (int x = 0; x < NSLOT && ok; ++x)
-                if (slots[x].active) ok = mbar_wait(&q_full[x], 0, abort_flag);
             tc_fence_after();
-            uint32_t seq = 0;
-            int stage_of[NSLOT][2];
-            for (int n = 0; n <= max_items && ok; ++n) {
-                for (int x = 0; x < NSLOT && ok; ++x) {
-                    if (n < slots[x].n_items) {
-                        const uint32_t s = seq % STAGES, ph = (seq / STAGES) & 1u;
-                        ++seq;
-                        if (!mbar_wait(&kv_full[s], ph, abort_flag)) { ok = false; break; }
-                        if (n > 0 && !mbar_wait(&s_free[x], (n - 1) & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t qa = smem_u32(sQ + x * tc::kTileBytes);
-                        const uint32_t ka = smem_u32(sKV + s * 2 * tc::kTileBytes);
+            const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dk0 = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+            const uint64_t dv0 = smem_desc_sw128(smem_u32(sKV + tc::kTileBytes), 16, 1024);
+            constexpr uint64_t kStageStep = (2 * tc::kTileBytes) >> 4;
+            // S(n) is issued as soon as its tile has landed and the softmax has read S(n-1),
+            // P.V(n-1) right after it, as soon as P(n-1) is in TMEM
+            for (int n = 0; n <= n_items && ok; ++n) {
+                if (n < n_items) {
+                    const uint32_t s = n % STAGES, ph = (n / STAGES) & 1u;
+                    if (!mbar_wait_warp(&kv_full[s], ph, abort_flag)) { ok = false; break; }
+                    if (n > 0 && !mbar_wait_warp(s_free, (n - 1) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    if (leader) {
+                        const uint64_t dk = dk0 + s * kStageStep;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_ss(tmem + Lay::colS(x), smem_desc_sw128(qa + 32 * kk, 16, 1024),
-                                    smem_desc_sw128(ka + 32 * kk, 16, 1024), tc::kIdescS, kk > 0);
-                        umma_commit(&s_full[x]);
-                        any_mma = true;
-                        stage_of[x][n & 1] = s;
+                            umma_ss(tmem + Lay::colS(x), dq + 2 * kk, dk + 2 * kk, tc::kIdescS, kk > 0);
+                        umma_commit(s_full);
                     }
-                    if (n >= 1 && n <= slots[x].n_items) {
-                        const int m = n - 1;
-                        if (!mbar_wait(&p_full[x], m & 1, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
-                        const int s = stage_of[x][m & 1];
-                        const uint32_t va = smem_u32(sKV + s * 2 * tc::kTileBytes + tc::kTileBytes);
+                    __syncwarp();
+                    any_mma = true;
+                }
+                if (n >= 1) {
+                    const int m = n - 1;
+                    const uint32_t s = m % STAGES;
+                    if (!mbar_wait_warp(p_full, m & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    if (leader) {
+                        const uint64_t dv = dv0 + s * kStageStep;
+                        // V^T is two 64-key swizzle atoms of 8 KB; a K=16 step is 32 bytes
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
                             umma_ts(tmem + Lay::colO(x), tmem + Lay::colP(x) + 8 * kk,
-                                    smem_desc_sw128(va + 2048 * kk, 1024, 1024), tc::kIdescPV,
+                                    dv + (uint64_t)((kk >> 2) * (8192 >> 4) + (kk & 3) * 2), tc::kIdescPV,
                                     (m > 0 || kk > 0));
                         umma_commit(&kv_empty[s]);
-                        umma_commit(&pv_done[x]);
+                        umma_commit(pv_done);
                     }
+                    __syncwarp();
                 }
             }
             // every MMA (and its commits) must be finished before TMEM is released
             if (any_mma) {
-                umma_commit(drain_bar);
+                if (leader) umma_commit(drain_bar);
+                __syncwarp();
                 tc::drain_wait(drain_bar, 0);
             }
         }
     } else {
         // ------------------------------------------------------------------ softmax group
-        const int x = sx;
-        const tc::Slot& sl = slots[x];
+        setmaxnreg_inc<Lay::kRegsSoftmax>();
+        const int st = threadIdx.x - 128 - 128 * x;  // 0..127
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -336,11 +398,19 @@ __global__ void __launch_bounds__(64 + 128 * NSLOT, 1) attn_tc_kernel(const __gr
         const uint32_t tO = tmem + Lay::colO(x) + lane_off;
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
+        int j_next = (!a.dense && sl.cnt > 0) ? __ldg(sl.list) : 0;  // list entry of the next item
+        int lm_ptr = 0;                                              // landmark chunks: list cursor
         for (int n = 0; n < sl.n_items; ++n) {
-            const tc::Item it = tc::get_item(a, sl, n);
-            if (!mbar_wait_warp(&s_full[x], n & 1, abort_flag)) { ok = false; break; }
+            const int j_cur = j_next;
+            if (!a.dense && n + 1 < sl.cnt) j_next = __ldg(sl.list + n + 1);  // one item ahead
+            const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
+            if (!mbar_wait_warp(s_full, n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            uint32_t s0[32], s1[32], s2[32], s3[32];
+            uint32_t sv[128];
+            uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv + 0);
+            uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv + 32);
+            uint32_t(&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv + 64);
+            uint32_t(&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv + 96);
             tmem_ld_32x32b_x32(tS + 0, s0);
             tmem_ld_32x32b_x32(tS + 32, s1);
             tmem_ld_32x32b_x32(tS + 64, s2);
@@ -350,88 +420,115 @@ __global__ void __launch_bounds__(64 + 128 * NSLOT, 1) attn_tc_kernel(const __gr
             reg_fence(s2);
             reg_fence(s3);
             tc_fence_before();
-            mbar_arrive(&s_free[x]);
+            mbar_arrive(s_free);
 
-            // logits in base-2 units, masked columns at -inf
-            float xs[128];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                xs[c] = __uint_as_float(s0[c]) * a.scale_log2;
-                xs[32 + c] = __uint_as_float(s1[c]) * a.scale_log2;
-                xs[64 + c] = __uint_as_float(s2[c]) * a.scale_log2;
-                xs[96 + c] = __uint_as_float(s3[c]) * a.scale_log2;
-            }
+            // Masked columns become -inf; landmark chunks add their per-column bias in base-2
+            // units (so their values are scaled here and `mul` becomes 1).
+            float mul = a.scale_log2;
             if (it.kind == 2) {
-                const float4* bp = reinterpret_cast<const float4*>(a.lbias2 + it.chunk * 128);
-                const uint32_t* mw = lmask + x * mask_words + it.chunk * 4;
+                // listed tiles of this chunk: the next run of the ascending list
+                uint32_t mw[4] = {0u, 0u, 0u, 0u};
+                const int c_lo = it.chunk * 128;
+                while (lm_ptr < sl.cnt) {
+                    const int j = __ldg(sl.list + lm_ptr);
+                    if (j >= c_lo + 128) break;
+                    if (j >= c_lo) mw[(j - c_lo) >> 5] |= 1u << (j & 31);
+                    ++lm_ptr;
+                }
+                const float4* bp = reinterpret_cast<const float4*>(a.lbias2 + c_lo);
 #pragma unroll
                 for (int c4 = 0; c4 < 32; ++c4) {
-                    const float4 b = __ldg(bp + c4);
-                    const int j = it.chunk * 128 + 4 * c4;
-                    const uint32_t word = (j >> 5) < mask_words ? mw[c4 >> 3] : 0u;
-                    const float bb[4] = {b.x, b.y, b.z, b.w};
+                    const float4 bv = __ldg(bp + c4);
+                    const uint32_t word = mw[c4 >> 3];
+                    const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const bool listed = (word >> ((4 * c4 + u) & 31)) & 1u;
-                        xs[4 * c4 + u] = listed ? -INFINITY : xs[4 * c4 + u] + bb[u];
+                        const int c = 4 * c4 + u;
+                        const bool listed = (word >> (c & 31)) & 1u;
+                        const float xv = fmaf(__uint_as_float(sv[c]), a.scale_log2, bb[u]);
+                        sv[c] = __float_as_uint(listed ? -INFINITY : xv);
                     }
                 }
-            } else {
+                mul = 1.0f;
+            } else if (it.lo > 0 || it.hi < 128) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (c < it.lo || c >= it.hi) xs[c] = -INFINITY;
+                    if (c < it.lo || c >= it.hi) sv[c] = __float_as_uint(-INFINITY);
             }
-            float mx = xs[0];
+            float mx8[8];
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, xs[c]);
+            for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sv[u]);
+#pragma unroll
+            for (int c = 8; c < 128; c += 16)
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    mx8[u] = fmax3(mx8[u], __uint_as_float(sv[c + u]), __uint_as_float(sv[c + 8 + u]));
+            const float mx_raw = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                       fmaxf(mx8[6], mx8[7]));
+            const float mx = mx_raw * mul;  // base-2 units (-inf stays -inf)
             float m_new = m_run;
             if (mx > m_run + 8.0f) m_new = mx;  // lazy max: rescale only on growth beyond 2^8
             const float m_use = m_new == -INFINITY ? 0.0f : m_new;
             const float alpha = ex2_approx(m_run - m_use);  // 0 on the first item
-            float sum = 0.0f;
+            // Ping-pong: the two slots take turns on the exponential units, so that one slot's
+            // exponentials overlap the other's TMEM round trips and barrier hand-offs.  Slot 0
+            // runs batch n after slot 1's batch n-1, slot 1 after slot 0's batch n; a slot that
+            // has finished (or given up) no longer holds the other back.
+            if (x == 1 || n > 0) {
+                const uint32_t par = (x == 0 ? (uint32_t)(n - 1) : (uint32_t)n) & 1u;
+                if (!tc::wait_token(&tok[x], par, &slot_done[1 - x], abort_flag)) { ok = false; break; }
+            }
+            const float2 mul2 = make_float2(mul, mul);
+            const float2 neg2 = make_float2(-m_use, -m_use);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
             uint32_t pk[64];
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-                const float p0 = ex2_approx(xs[2 * c] - m_use);
-                const float p1 = ex2_approx(xs[2 * c + 1] - m_use);
-                sum += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
+                const float2 xv =
+                    __ffma2_rn(make_float2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), mul2, neg2);
+                float2 p;
+                if ((c & 7) >= 8 - SA_EXP2_FMA_PAIRS_PER8) {
+                    p = exp2_poly2(xv);  // FMA pipe: takes load off the MUFU
+                } else {
+                    p.x = ex2_approx(xv.x);
+                    p.y = ex2_approx(xv.y);
+                }
+                acc[c & 3] = __fadd2_rn(acc[c & 3], p);
+                pk[c] = pack_bf16x2(p.x, p.y);
             }
+            mbar_arrive(&tok[1 - x]);  // the other slot may start its next batch
+            const float2 acc_all = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+            l_run = l_run * alpha + (acc_all.x + acc_all.y);
+            m_run = m_new;
             if (n > 0) {
-                // the previous P.V product must be done before O is rescaled or P overwritten
-                if (!mbar_wait_warp(&pv_done[x], (n - 1) & 1, abort_flag)) { ok = false; break; }
+                // the previous P.V product must be done before O is rescaled or P overwritten;
+                // the exponentials above overlap with it
+                if (!mbar_wait_warp(pv_done, (n - 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                    uint32_t o0[32], o1[32];
-                    tmem_ld_32x32b_x32(tO + 0, o0);
-                    tmem_ld_32x32b_x32(tO + 32, o1);
-                    tmem_ld_wait(o0);
-                    reg_fence(o1);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        o0[c] = __float_as_uint(__uint_as_float(o0[c]) * alpha);
-                        o1[c] = __float_as_uint(__uint_as_float(o1[c]) * alpha);
+                    for (int c = 0; c < 64; c += 16) {
+                        uint32_t ov[16];
+                        tmem_ld_32x32b_x16(tO + c, ov);
+                        tmem_ld_wait16(ov);
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * alpha);
+                        tmem_st_32x32b_x16(tO + c, ov);
                     }
-                    tmem_st_32x32b_x32(tO + 0, o0);
-                    tmem_st_32x32b_x32(tO + 32, o1);
                 }
             }
-            l_run = l_run * alpha + sum;
-            m_run = m_new;
-            uint32_t pa[32], pb[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                pa[c] = pk[c];
-                pb[c] = pk[32 + c];
-            }
+            uint32_t(&pa)[32] = *reinterpret_cast<uint32_t(*)[32]>(pk + 0);
+            uint32_t(&pb)[32] = *reinterpret_cast<uint32_t(*)[32]>(pk + 32);
             tmem_st_32x32b_x32(tP + 0, pa);
             tmem_st_32x32b_x32(tP + 32, pb);
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&p_full[x]);
+            mbar_arrive(p_full);
         }
+        slot_done[x] = 1;  // from here on this slot no longer takes turns
         // ---- epilogue: O / l, LSE, store valid rows
-        if (ok && sl.n_items > 0 && mbar_wait_warp(&pv_done[x], (sl.n_items - 1) & 1, abort_flag)) {
+        if (ok && sl.n_items > 0 && mbar_wait_warp(pv_done, (sl.n_items - 1) & 1, abort_flag)) {
             tc_fence_after();
             uint32_t o0[32], o1[32];
             tmem_ld_32x32b_x32(tO + 0, o0);
@@ -465,6 +562,12 @@ __global__ void __launch_bounds__(64 + 128 * NSLOT, 1) attn_tc_kernel(const __gr
                         l_run > 0.0f ? (m_fin + log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
                 }
             }
+        } else if (ok && sl.active && sl.n_items == 0 && r < sl.nq) {
+            // nothing to attend: zero output, LSE = -inf
+            uint4* dst = reinterpret_cast<uint4*>(a.o + ((int64_t)sl.qrow + r) * 64);
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) dst[c8] = make_uint4(0, 0, 0, 0);
+            if (a.lse) a.lse[(int64_t)sl.qrow + r] = -INFINITY;
         }
         // report skipped list entries once per slot
         if (ok && st == 0 && !a.dense)

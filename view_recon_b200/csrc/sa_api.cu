@@ -5,6 +5,7 @@
 #include <mutex>
 #include <string.h>
 
+#include "k_attn_prep.cuh"
 #include "k_attn_simt.cuh"
 #include "k_attn_tc.cuh"
 #include "k_pool.cuh"
@@ -14,7 +15,7 @@
 namespace {
 
 constexpr int kTcSlots = 2;
-constexpr int kTcStages = 5;
+constexpr int kTcStages = 3;  // per slot
 constexpr int kMaxDevices = 64;
 
 struct Geo {
@@ -76,6 +77,7 @@ sa_status launch_status() {
 // ---- per-device one-time kernel attributes
 std::mutex g_attr_mu;
 bool g_attr_done[kMaxDevices];
+bool g_tc_regs_ok[kMaxDevices];
 
 sa_status ensure_attributes() {
     int dev = 0;
@@ -96,10 +98,16 @@ sa_status ensure_attributes() {
                                200 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SEL_MAX_NT * 4) == cudaSuccess;
+    // The tensor-core kernel moves registers between its warpgroups (setmaxnreg); that is only
+    // satisfiable if the block is launched with at least the registers the split hands out.
+    cudaFuncAttributes fa;
+    ok &= cudaFuncGetAttributes(&fa, attn_tc_kernel<kTcSlots, kTcStages>) == cudaSuccess;
+    using Lay = TcLayout<kTcSlots, kTcStages>;
     if (!ok) {
         cudaGetLastError();
         return SA_ERR_CUDA;
     }
+    g_tc_regs_ok[dev] = (uint32_t)fa.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded;
     g_attr_done[dev] = true;
     return SA_OK;
 }
@@ -125,31 +133,60 @@ EncodeTiledFn encoder() {
     return g_encode;
 }
 
-// [rows][64] bf16 matrix, 128-row boxes with the 128-byte swizzle.
-bool encode_rows_bf16(CUtensorMap* m, const void* base, int64_t rows) {
+// [rows][cols] bf16 matrix with (box_cols x box_rows) boxes and the 128-byte swizzle
+// (box_cols * 2 bytes must be 128).
+bool encode_bf16_2d(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, uint32_t box_cols,
+                    uint32_t box_rows) {
     EncodeTiledFn enc = encoder();
-    if (!enc || rows < 1) return false;
-    const cuuint64_t dims[2] = {64, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {128};
-    const cuuint32_t box[2] = {64, 128};
+    if (!enc || rows < 1 || cols < 1) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows][64] bf16 matrix read in 128-row boxes (Q, K, sink keys, landmark keys).
+bool encode_rows_bf16(CUtensorMap* m, const void* base, int64_t rows) {
+    return encode_bf16_2d(m, base, 64, rows, 64, 128);
+}
+
+// Transposed V tiles: [tiles * 64][128] bf16 read as two 64 x 64 boxes per tile.
+bool encode_vt_tiles(CUtensorMap* m, const void* base, int64_t tiles) {
+    return encode_bf16_2d(m, base, 128, tiles * 64, 64, 64);
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct LandmarkWs {
-    size_t lk, lv, bias, total;
+// Workspace of the tensor-core attention call (all offsets 256-byte aligned):
+//   vt   transposed V tiles of every key tile [bh][n_vtiles][64][128] bf16
+//   svt  transposed V tiles of the sink segment [bh][n_sink_tiles][64][128]
+//   lk   landmark key table [bh][ntp][64] bf16, lvt its transposed value tiles, lbias [ntp] f32
+struct AttnWs {
+    int64_t n_vtiles, n_sink_tiles, n_lm_chunks, ntp;
+    size_t vt, svt, lk, lvt, lbias, total;
 };
-LandmarkWs landmark_ws(const Geo& g) {
-    const int64_t ntp = (g.nt + 127) / 128 * 128;
-    LandmarkWs w;
-    w.lk = 0;
-    w.lv = align256((size_t)g.bh * ntp * 64 * 2);
-    w.bias = w.lv + align256((size_t)g.bh * ntp * 64 * 2);
-    w.total = w.bias + align256((size_t)ntp * 4);
+AttnWs attn_ws(const Geo& g, bool dense, bool landmark) {
+    AttnWs w;
+    constexpr size_t kTile = 64 * 128 * 2;
+    w.ntp = (g.nt + 127) / 128 * 128;
+    w.n_vtiles = dense ? (g.L + 127) / 128 : g.nt;
+    w.n_sink_tiles = dense ? 0 : (g.S * g.n_sink + 127) / 128;
+    w.n_lm_chunks = (!dense && landmark) ? w.ntp / 128 : 0;
+    size_t off = 0;
+    w.vt = off;
+    off += align256((size_t)g.bh * w.n_vtiles * kTile);
+    w.svt = off;
+    off += align256((size_t)g.bh * w.n_sink_tiles * kTile);
+    w.lk = off;
+    off += (!dense && landmark) ? align256((size_t)g.bh * w.ntp * 64 * 2) : 0;
+    w.lvt = off;
+    off += align256((size_t)g.bh * w.n_lm_chunks * kTile);
+    w.lbias = off;
+    off += (!dense && landmark) ? align256((size_t)w.ntp * 4) : 0;
+    w.total = off;
     return w;
 }
 
@@ -171,33 +208,56 @@ sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v,
     if (use_tc(g)) {
         TcArgs a;
         memset(&a, 0, sizeof(a));
-        const int64_t ntp = (g.nt + 127) / 128 * 128;
+        const AttnWs w = attn_ws(g, dense, landmark != 0);
+        if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
+        uint8_t* base = static_cast<uint8_t*>(ws);
         const int64_t n_sink_rows = g.S * g.n_sink;
         bool ok = encode_rows_bf16(&a.tm_q, q, g.bh * g.L) && encode_rows_bf16(&a.tm_k, k, g.bh * g.L) &&
-                  encode_rows_bf16(&a.tm_v, v, g.bh * g.L);
-        if (!dense && n_sink_rows > 0)
+                  encode_vt_tiles(&a.tm_vt, base + w.vt, g.bh * w.n_vtiles);
+        if (w.n_sink_tiles > 0)
             ok = ok && encode_rows_bf16(&a.tm_sk, sink_k, g.bh * n_sink_rows) &&
-                 encode_rows_bf16(&a.tm_sv, sink_v, g.bh * n_sink_rows);
+                 encode_vt_tiles(&a.tm_svt, base + w.svt, g.bh * w.n_sink_tiles);
         else
-            a.tm_sk = a.tm_k, a.tm_sv = a.tm_v;
-        LandmarkWs lw = landmark_ws(g);
-        if (!dense && landmark) {
-            uint8_t* base = static_cast<uint8_t*>(ws);
-            ok = ok && encode_rows_bf16(&a.tm_lk, base + lw.lk, g.bh * ntp) &&
-                 encode_rows_bf16(&a.tm_lv, base + lw.lv, g.bh * ntp);
-            a.lbias2 = reinterpret_cast<const float*>(base + lw.bias);
+            a.tm_sk = a.tm_k, a.tm_svt = a.tm_vt;
+        if (w.n_lm_chunks > 0) {
+            ok = ok && encode_rows_bf16(&a.tm_lk, base + w.lk, g.bh * w.ntp) &&
+                 encode_vt_tiles(&a.tm_lvt, base + w.lvt, g.bh * w.n_lm_chunks);
+            a.lbias2 = reinterpret_cast<const float*>(base + w.lbias);
         } else {
-            a.tm_lk = a.tm_k, a.tm_lv = a.tm_v;
+            a.tm_lk = a.tm_k, a.tm_lvt = a.tm_vt;
         }
         if (!ok) return SA_ERR_CUDA;
-        if (!dense && landmark) {
-            uint8_t* base = static_cast<uint8_t*>(ws);
-            const int64_t n4 = g.bh * ntp * 16;
+        // operand preparation: transposed V tiles (and the landmark tables)
+        {
+            VtArgs t;
+            t.src = static_cast<const __nv_bfloat16*>(v);
+            t.dst = reinterpret_cast<__nv_bfloat16*>(base + w.vt);
+            t.tiles_per_head = (int32_t)w.n_vtiles;
+            t.frame_mode = dense ? 0 : 1;
+            t.tokens = (int32_t)g.N;
+            t.tpf = (int32_t)g.tpf;
+            t.L = (int32_t)g.L;
+            t.rows_per_head = (int32_t)g.L;
+            if (w.n_vtiles > 2147483647 || g.bh > 65535) return SA_ERR_UNSUPPORTED;
+            vtile_transpose_kernel<<<dim3((unsigned)w.n_vtiles, (unsigned)g.bh), 256, 0, stream>>>(t);
+            if ((st = launch_status()) != SA_OK) return st;
+            if (w.n_sink_tiles > 0) {
+                t.src = static_cast<const __nv_bfloat16*>(sink_v);
+                t.dst = reinterpret_cast<__nv_bfloat16*>(base + w.svt);
+                t.tiles_per_head = (int32_t)w.n_sink_tiles;
+                t.frame_mode = 0;
+                t.rows_per_head = (int32_t)n_sink_rows;
+                vtile_transpose_kernel<<<dim3((unsigned)w.n_sink_tiles, (unsigned)g.bh), 256, 0, stream>>>(t);
+                if ((st = launch_status()) != SA_OK) return st;
+            }
+        }
+        if (w.n_lm_chunks > 0) {
+            const int64_t n4 = g.bh * w.ntp * 16;
             const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 148 * 32);
             landmark_prep_kernel<<<blocks, 256, 0, stream>>>(
-                k_pool, v_pool, k_cnt, reinterpret_cast<__nv_bfloat16*>(base + lw.lk),
-                reinterpret_cast<__nv_bfloat16*>(base + lw.lv), reinterpret_cast<float*>(base + lw.bias),
-                (int32_t)g.bh, (int32_t)g.nt, (int32_t)ntp);
+                k_pool, v_pool, k_cnt, reinterpret_cast<__nv_bfloat16*>(base + w.lk),
+                reinterpret_cast<__nv_bfloat16*>(base + w.lvt), reinterpret_cast<float*>(base + w.lbias),
+                (int32_t)g.bh, (int32_t)g.nt, (int32_t)w.ntp);
             if ((st = launch_status()) != SA_OK) return st;
         }
         a.kept_idx = kept_idx;
@@ -211,18 +271,27 @@ sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v,
         a.tpf = (int32_t)g.tpf;
         a.nt = (int32_t)g.nt;
         a.L = (int32_t)g.L;
-        a.ntp = (int32_t)ntp;
+        a.ntp = (int32_t)w.ntp;
+        a.n_vtiles = (int32_t)w.n_vtiles;
         a.n_sink_rows = (int32_t)n_sink_rows;
-        a.n_sink_tiles = dense ? 0 : (int32_t)((n_sink_rows + 127) / 128);
-        a.n_lm_chunks = (!dense && landmark) ? (int32_t)(ntp / 128) : 0;
+        a.n_sink_tiles = (int32_t)w.n_sink_tiles;
+        a.n_lm_chunks = (int32_t)w.n_lm_chunks;
         a.dense = dense ? 1 : 0;
-        a.landmark = (!dense && landmark) ? 1 : 0;
+        a.landmark = w.n_lm_chunks > 0 ? 1 : 0;
         a.q_per_head = dense ? (int32_t)((g.L + 127) / 128) : (int32_t)g.nt;
         a.total_items = (int32_t)(g.bh * a.q_per_head);
         a.scale_log2 = (float)((double)g.scale * 1.4426950408889634);
         using Lay = TcLayout<kTcSlots, kTcStages>;
-        const int mask_words = a.landmark ? (a.nt + 31) / 32 : 0;
-        const size_t smem = Lay::smem_bytes(mask_words);
+        {
+            int dev = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+            if (!g_tc_regs_ok[dev]) return SA_ERR_UNSUPPORTED;
+        }
+        // exact division by tpf with a multiply-high, checked for every tile index
+        a.tpf_magic = (uint32_t)((0x100000000ull + (uint64_t)g.tpf - 1) / (uint64_t)g.tpf);
+        for (int64_t j = 0; j < g.nt; ++j)
+            if ((int64_t)(((uint64_t)j * a.tpf_magic) >> 32) != j / g.tpf) return SA_ERR_UNSUPPORTED;
+        const size_t smem = Lay::smem_bytes();
         if (smem > 227 * 1024) return SA_ERR_UNSUPPORTED;
         const int grid = (a.total_items + kTcSlots - 1) / kTcSlots;
         attn_tc_kernel<kTcSlots, kTcStages><<<grid, Lay::kThreads, smem, stream>>>(a);
@@ -469,8 +538,15 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, con
 size_t sa_sparse_attn_workspace_size(const sa_shape* shape, int32_t landmark) {
     Geo g;
     if (geo_of(shape, &g) != SA_OK) return 0;
-    if (!landmark || !use_tc(g)) return 0;
-    return landmark_ws(g).total;
+    if (!use_tc(g)) return 0;
+    return attn_ws(g, false, landmark != 0).total;
+}
+
+size_t sa_dense_attn_workspace_size(const sa_shape* shape) {
+    Geo g;
+    if (geo_of(shape, &g) != SA_OK) return 0;
+    if (!use_tc(g)) return 0;
+    return attn_ws(g, true, false).total;
 }
 
 sa_status sa_sparse_attn_fwd(const sa_shape* shape, const void* q, const void* k, const void* v,
@@ -494,26 +570,29 @@ sa_status sa_sparse_attn_fwd(const sa_shape* shape, const void* q, const void* k
         if (!k_pool_or_null || !v_pool_or_null || !k_cnt_or_null || !aligned16(k_pool_or_null) ||
             !aligned16(v_pool_or_null) || !aligned16(k_cnt_or_null))
             return SA_ERR_INVALID_ARG;
-        if (g.nt > 16384) return SA_ERR_UNSUPPORTED;
-        const size_t need = sa_sparse_attn_workspace_size(shape, 1);
-        if (need && (!workspace_or_null || workspace_bytes < need || !aligned16(workspace_or_null)))
-            return SA_ERR_WORKSPACE;
     }
+    const size_t need = sa_sparse_attn_workspace_size(shape, landmark);
+    if (need && (!workspace_or_null || workspace_bytes < need || !aligned16(workspace_or_null)))
+        return SA_ERR_WORKSPACE;
     return attn_common(g, q, k, v, kept_idx, kept_cnt, max_kept, sink_k_or_null, sink_v_or_null, landmark ? 1 : 0,
                        k_pool_or_null, v_pool_or_null, k_cnt_or_null, workspace_or_null, workspace_bytes, o,
                        lse_or_null, false, stream);
 }
 
-sa_status sa_dense_attn_fwd(const sa_shape* shape, const void* q, const void* k, const void* v, void* o,
-                            float* lse_or_null, sa_stream_t stream) {
+sa_status sa_dense_attn_fwd(const sa_shape* shape, const void* q, const void* k, const void* v,
+                            void* workspace_or_null, size_t workspace_bytes, void* o, float* lse_or_null,
+                            sa_stream_t stream) {
     Geo g;
     sa_status st = geo_of(shape, &g);
     if (st != SA_OK) return st;
     if (!q || !k || !v || !o) return SA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse_or_null && !aligned16(lse_or_null)))
         return SA_ERR_INVALID_ARG;
-    return attn_common(g, q, k, v, nullptr, nullptr, 0, nullptr, nullptr, 0, nullptr, nullptr, nullptr, nullptr, 0,
-                       o, lse_or_null, true, stream);
+    const size_t need = sa_dense_attn_workspace_size(shape);
+    if (need && (!workspace_or_null || workspace_bytes < need || !aligned16(workspace_or_null)))
+        return SA_ERR_WORKSPACE;
+    return attn_common(g, q, k, v, nullptr, nullptr, 0, nullptr, nullptr, 0, nullptr, nullptr, nullptr,
+                       workspace_or_null, workspace_bytes, o, lse_or_null, true, stream);
 }
 
 }  // extern "C"

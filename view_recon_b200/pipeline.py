@@ -118,8 +118,12 @@ class SparseGlobalAttention:
         else:
             n += 2  # scores + select
         n += 1  # attention
-        if self.landmark and sa.sa_sparse_attn_workspace_size(self.shape, True) > 0:
-            n += 1  # landmark tables
+        if sa.sa_sparse_attn_workspace_size(self.shape, self.landmark) > 0:
+            n += 1  # transposed V tiles
+            if self.frames * self.shape.n_sink > 0:
+                n += 1  # transposed sink V tiles
+            if self.landmark:
+                n += 1  # landmark tables
         return n
 
 
@@ -130,5 +134,25 @@ def dense_attention(q, k, v, frames: int, tokens: int, dtype: str = "bf16", with
     shp = sa.shape(bh, frames, tokens, q.shape[2], 128, 0, dtype)
     o = torch.empty_like(q)
     lse = torch.empty((bh, frames * tokens), dtype=torch.float32, device=q.device) if with_lse else None
-    sa.sa_dense_attn_fwd(shp, q, k, v, o, lse, stream)
+    nbytes = sa.sa_dense_attn_workspace_size(shp)
+    ws = torch.empty((nbytes,), dtype=torch.uint8, device=q.device) if nbytes else None
+    sa.sa_dense_attn_fwd(shp, q, k, v, ws, o, lse, stream)
     return o, lse
+
+
+class DenseAttention:
+    """Dense control with its workspace allocated once (for repeated calls at one shape)."""
+
+    def __init__(self, bh: int, frames: int, tokens: int, dtype: str = "bf16", head_dim: int = 64, device=None):
+        import torch
+        self.shape = sa.shape(bh, frames, tokens, head_dim, 128, 0, dtype)
+        dev = torch.device(device if device is not None else "cuda")
+        nbytes = sa.sa_dense_attn_workspace_size(self.shape)
+        self.ws = torch.empty((nbytes,), dtype=torch.uint8, device=dev) if nbytes else None
+        tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.o = torch.empty((bh, frames * tokens, head_dim), dtype=tdt, device=dev)
+        self.lse = torch.empty((bh, frames * tokens), dtype=torch.float32, device=dev)
+
+    def __call__(self, q, k, v, stream=None):
+        sa.sa_dense_attn_fwd(self.shape, q, k, v, self.ws, self.o, self.lse, stream)
+        return self.o, self.lse

@@ -28,7 +28,8 @@ SA_BF16 = 1
 # every symbol include/sa.h declares
 EXPORTS = [
     "sa_num_tiles", "sa_max_kept", "sa_tile_pool", "sa_tile_scores", "sa_select_workspace_size",
-    "sa_select_topk", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_fwd",
+    "sa_select_topk", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
+    "sa_dense_attn_fwd",
     "sa_status_string", "sa_check_device_error", "sa_set_wait_limit_ns",
 ]
 
@@ -76,7 +77,8 @@ def load(path: str | None = None):
         "sa_sparse_attn_workspace_size": (sz, [shp, i32]),
         "sa_sparse_attn_fwd": (i32, [shp, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp, vp,
                                      vp]),
-        "sa_dense_attn_fwd": (i32, [shp, vp, vp, vp, vp, vp, vp]),
+        "sa_dense_attn_workspace_size": (sz, [shp]),
+        "sa_dense_attn_fwd": (i32, [shp, vp, vp, vp, vp, sz, vp, vp, vp]),
         "sa_status_string": (ctypes.c_char_p, [i32]),
         "sa_check_device_error": (i32, [vp]),
         "sa_set_wait_limit_ns": (i32, [ctypes.c_int64]),
@@ -171,9 +173,14 @@ def sa_sparse_attn_fwd(shp, q, k, v, kept_idx, kept_cnt, max_kept, sink_k, sink_
     _check("sa_sparse_attn_fwd", st)
 
 
-def sa_dense_attn_fwd(shp, q, k, v, o, lse=None, stream=None):
-    st = load().sa_dense_attn_fwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                  _stream(stream))
+def sa_dense_attn_workspace_size(shp) -> int:
+    return int(load().sa_dense_attn_workspace_size(ctypes.byref(shp)))
+
+
+def sa_dense_attn_fwd(shp, q, k, v, workspace, o, lse=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().sa_dense_attn_fwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(workspace), ws_bytes, _ptr(o),
+                                  _ptr(lse), _stream(stream))
     _check("sa_dense_attn_fwd", st)
 
 
