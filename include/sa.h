@@ -146,6 +146,26 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null,
                          int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
                          void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream);
 
+/*
+ * sa_select_topk in streamed mode without any caller-provided memory.  No passage of the
+ * pages corresponds to this call; it exists for callers that cannot allocate device memory
+ * where this step runs - for instance plugin code inside a host framework that owns the
+ * device memory pool and hands out no allocator, or a latency-bound loop that forbids
+ * allocation after start-up.  Instead of a workspace it uses a fixed 8 MiB scratch array that
+ * is part of the library image: every GPU that loads the library holds it until the process
+ * exits.  The result is the same as sa_select_topk(shape, NULL, q_pool, k_pool, k, ...).
+ *   Limit: nt <= 32768 (the scratch holds at least 64 whole score rows); larger shapes
+ *          return SA_ERR_UNSUPPORTED.
+ *   Set-up: the first call on a device looks up the scratch array's device address (a host-
+ *          side runtime query); make that first call before any stream capture begins.
+ *   Sharing: all calls on a device use the same array and it keeps the last call's contents
+ *          (every score row is written before it is read, so nothing needs clearing).  Calls
+ *          whose kernels overlap on the GPU (e.g. on different streams) race on it.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine is called.
+ */
+sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, const float* k_pool, int32_t k,
+                                 int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept, sa_stream_t stream);
+
 /* Bytes of workspace sa_sparse_attn_fwd needs: on the tensor-core path (bf16, tile 128) a
  * transposed copy of every V tile it may gather (the size of V plus the sink segment) and, in
  * landmark mode, the bf16 landmark tables; 0 on the CUDA-core path (f32 or tile 64). */

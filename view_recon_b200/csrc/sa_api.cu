@@ -12,6 +12,10 @@
 #include "k_scores.cuh"
 #include "k_select.cuh"
 
+// Fixed scratch of sa_select_topk_noalloc: one block of score rows (2 Mi floats = 8 MiB).
+constexpr long long kNoallocScratchFloats = 1ll << 21;
+static __device__ __align__(256) float g_sa_noalloc_scores[kNoallocScratchFloats];
+
 namespace {
 
 constexpr int kTcSlots = 2;
@@ -109,6 +113,28 @@ sa_status ensure_attributes() {
     }
     g_tc_regs_ok[dev] = (uint32_t)fa.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded;
     g_attr_done[dev] = true;
+    return SA_OK;
+}
+
+// ---- fixed scratch for sa_select_topk_noalloc: one block of score rows (8 MiB), part of the
+// library image on every device that loads it; its device address is looked up once per device.
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices];
+
+sa_status noalloc_scratch(float** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_sa_noalloc_scores) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return SA_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
     return SA_OK;
 }
 
@@ -508,6 +534,58 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, con
     // streamed: score one L2-resident block of rows at a time, then select from it
     const int64_t R = (int64_t)select_rows_per_block(g);
     float* blk = static_cast<float*>(workspace_or_null);
+    for (int64_t h = 0; h < g.bh; ++h) {
+        for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
+            const int64_t rows = std::min<int64_t>(R, g.nt - i0);
+            ScoreArgs sc;
+            sc.q_pool = q_pool;
+            sc.k_pool = k_pool;
+            sc.out = blk;
+            sc.ldo = g.nt;
+            sc.nt = (int32_t)g.nt;
+            sc.h0 = (int32_t)h;
+            sc.i0 = (int32_t)i0;
+            sc.rows = (int32_t)rows;
+            tile_scores_kernel<<<dim3((unsigned)((g.nt + 63) / 64), (unsigned)((rows + 63) / 64), 1), 256, 0,
+                                 stream>>>(sc);
+            if ((st = launch_status()) != SA_OK) return st;
+            a.scores = blk;
+            a.lds = g.nt;
+            a.h0 = (int32_t)h;
+            a.i0 = (int32_t)i0;
+            a.rows = (int32_t)rows;
+            select_topk_kernel<<<dim3((unsigned)rows, 1), SEL_THREADS, smem, stream>>>(a);
+            if ((st = launch_status()) != SA_OK) return st;
+        }
+    }
+    return SA_OK;
+}
+
+sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, const float* k_pool, int32_t k,
+                                 int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept, sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    if (k < 0 || !kept_idx || !kept_cnt || !aligned16(kept_idx) || !aligned16(kept_cnt)) return SA_ERR_INVALID_ARG;
+    if (!q_pool || !k_pool || !aligned16(q_pool) || !aligned16(k_pool)) return SA_ERR_INVALID_ARG;
+    if (max_kept < max_kept_of(g, k)) return SA_ERR_INVALID_ARG;
+    // the fixed scratch must hold at least 64 whole score rows
+    if (g.nt > SEL_MAX_NT || g.nt * 64 > kNoallocScratchFloats) return SA_ERR_UNSUPPORTED;
+    if ((st = ensure_attributes()) != SA_OK) return st;
+    float* blk = nullptr;
+    if ((st = noalloc_scratch(&blk)) != SA_OK) return st;
+    const int64_t R = std::min<int64_t>(g.nt, (kNoallocScratchFloats / g.nt) / 64 * 64);
+    SelectArgs a;
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.nt = (int32_t)g.nt;
+    a.tpf = (int32_t)g.tpf;
+    a.tile = (int32_t)g.T;
+    a.tokens = (int32_t)g.N;
+    a.n_sink = (int32_t)g.n_sink;
+    a.k = k;
+    a.max_kept = max_kept;
+    const size_t smem = (size_t)g.nt * 4;
     for (int64_t h = 0; h < g.bh; ++h) {
         for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
             const int64_t rows = std::min<int64_t>(R, g.nt - i0);

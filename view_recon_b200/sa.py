@@ -28,7 +28,7 @@ SA_BF16 = 1
 # every symbol include/sa.h declares
 EXPORTS = [
     "sa_num_tiles", "sa_max_kept", "sa_tile_pool", "sa_tile_scores", "sa_select_workspace_size",
-    "sa_select_topk", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
+    "sa_select_topk", "sa_select_topk_noalloc", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
     "sa_dense_attn_fwd",
     "sa_status_string", "sa_check_device_error", "sa_set_wait_limit_ns",
 ]
@@ -74,6 +74,7 @@ def load(path: str | None = None):
         "sa_tile_scores": (i32, [shp, vp, vp, vp, vp]),
         "sa_select_workspace_size": (sz, [shp, i32]),
         "sa_select_topk": (i32, [shp, vp, vp, vp, i32, vp, vp, i32, vp, sz, vp]),
+        "sa_select_topk_noalloc": (i32, [shp, vp, vp, i32, vp, vp, i32, vp]),
         "sa_sparse_attn_workspace_size": (sz, [shp, i32]),
         "sa_sparse_attn_fwd": (i32, [shp, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp, vp,
                                      vp]),
@@ -157,6 +158,12 @@ def sa_select_topk(shp, scores, q_pool, k_pool, k, kept_idx, kept_cnt, max_kept,
                                _ptr(kept_idx), _ptr(kept_cnt), int(max_kept), _ptr(workspace), ws_bytes,
                                _stream(stream))
     _check("sa_select_topk", st)
+
+
+def sa_select_topk_noalloc(shp, q_pool, k_pool, k, kept_idx, kept_cnt, max_kept, stream=None):
+    st = load().sa_select_topk_noalloc(ctypes.byref(shp), _ptr(q_pool), _ptr(k_pool), int(k), _ptr(kept_idx),
+                                       _ptr(kept_cnt), int(max_kept), _stream(stream))
+    _check("sa_select_topk_noalloc", st)
 
 
 def sa_sparse_attn_workspace_size(shp, landmark: bool) -> int:
