@@ -224,6 +224,15 @@ sa_status sa_check_device_error(sa_stream_t stream);
  * with SA_ERR_TIMEOUT recorded; outputs of that launch are then undefined. */
 sa_status sa_set_wait_limit_ns(int64_t limit_ns);
 
+/* Test facility for the failure path (not for production use): while enable != 0, later
+ * launches of the tensor-core attention kernel (bf16, tile 128) on the current device never
+ * issue the first query-tile load of their first CTA, so that CTA's MMA warp waits for data
+ * that cannot arrive.  The wait runs out after the wait limit, the CTA drains what it has in
+ * flight and exits, and sa_check_device_error reports SA_ERR_TIMEOUT; the outputs of such a
+ * launch are undefined and the device stays usable.  Returns SA_ERR_CUDA if the setting
+ * cannot be written. */
+sa_status sa_test_withhold_query_load(int32_t enable);
+
 #ifdef __cplusplus
 }
 #endif

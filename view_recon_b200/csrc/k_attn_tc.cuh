@@ -161,10 +161,12 @@ __device__ __forceinline__ Item get_item_j(const TcArgs& a, const Slot& s, int n
     return it;
 }
 
-// Bounded wait that ignores the abort flag (used only to drain in-flight work).
+// Bounded wait that ignores the abort flag (used only to drain in-flight work).  Copies and
+// MMAs already issued complete in microseconds; the limit is at least 1 s whatever the
+// caller's wait limit, so that a CTA never exits with work of its own still in flight.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = sa_globaltimer();
-    const uint64_t limit = g_sa_wait_limit_ns;
+    const uint64_t limit = max(g_sa_wait_limit_ns, 1000000000ull);
     while (!mbar_test(bar, parity)) {
         if (sa_globaltimer() - t0 > limit) {
             sa_flag_error(SA_ERR_TIMEOUT);
@@ -304,7 +306,8 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             const bool leader = tc::elect_one();
             uint32_t issued_mask = 0, phase_mask = 0;  // per ring stage: a load was issued / its parity
             bool ok = true;
-            if (n_items > 0 && leader) {
+            const bool withhold = g_sa_test_withhold != 0 && blockIdx.x == 0 && x == 0;
+            if (n_items > 0 && leader && !withhold) {
                 mbar_arrive_expect_tx(q_full, tc::kTileBytes);
                 tma_load_2d(sQ, &a.tm_q, q_full, 0, sl.qrow);
             }
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             if (!ok) {  // let every copy this warp started land before the CTA exits
                 for (int s = 0; s < STAGES; ++s)
                     if ((issued_mask >> s) & 1u) tc::drain_wait(&kv_full[s], (phase_mask >> s) & 1u);
-                if (n_items > 0) tc::drain_wait(q_full, 0);
+                if (n_items > 0 && !withhold) tc::drain_wait(q_full, 0);
             }
         } else {
             // -------------------------------------------------------------- MMA issuer (slot x)

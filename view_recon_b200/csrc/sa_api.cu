@@ -101,7 +101,7 @@ sa_status ensure_attributes() {
     ok &= cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                200 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SEL_MAX_NT * 4) == cudaSuccess;
+                               (int)select_smem_bytes(SEL_MAX_NT)) == cudaSuccess;
     // The tensor-core kernel moves registers between its warpgroups (setmaxnreg); that is only
     // satisfiable if the block is launched with at least the registers the split hands out.
     cudaFuncAttributes fa;
@@ -420,6 +420,15 @@ sa_status sa_set_wait_limit_ns(int64_t limit_ns) {
     return SA_OK;
 }
 
+sa_status sa_test_withhold_query_load(int32_t enable) {
+    const int v = enable ? 1 : 0;
+    if (cudaMemcpyToSymbol(g_sa_test_withhold, &v, sizeof(v)) != cudaSuccess) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    return SA_OK;
+}
+
 sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, const void* v_or_null,
                        float* q_pool, float* k_pool, float* v_pool_or_null, int32_t* k_cnt, void* sink_k_or_null,
                        void* sink_v_or_null, sa_stream_t stream) {
@@ -521,7 +530,7 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, con
     a.n_sink = (int32_t)g.n_sink;
     a.k = k;
     a.max_kept = max_kept;
-    const size_t smem = (size_t)g.nt * 4;
+    const size_t smem = select_smem_bytes((int)g.nt);
     if (scores_or_null) {
         a.scores = scores_or_null;
         a.lds = g.nt;
@@ -585,7 +594,7 @@ sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, con
     a.n_sink = (int32_t)g.n_sink;
     a.k = k;
     a.max_kept = max_kept;
-    const size_t smem = (size_t)g.nt * 4;
+    const size_t smem = select_smem_bytes((int)g.nt);
     for (int64_t h = 0; h < g.bh; ++h) {
         for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
             const int64_t rows = std::min<int64_t>(R, g.nt - i0);

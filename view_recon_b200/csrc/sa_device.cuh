@@ -15,6 +15,9 @@
 __device__ int g_sa_error = 0;
 // Upper bound on any single device-side wait, in globaltimer nanoseconds.
 __device__ unsigned long long g_sa_wait_limit_ns = 2000000000ull;
+// Test facility (sa_test_withhold_query_load): when nonzero, CTA 0 of the tensor-core attention
+// kernel never issues its first query-tile load, so one wait can only end by running out.
+__device__ int g_sa_test_withhold = 0;
 
 __device__ __forceinline__ void sa_flag_error(int code) { atomicCAS(&g_sa_error, 0, code); }
 
@@ -100,6 +103,21 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 // 2-D tiled load of one box into shared memory, completing `bytes` on `bar`.
 // x (the innermost coordinate) is always 0 here, so the 16-byte rule holds; y may run past
 // the tensor's end, where the box is zero filled.
+// Order generic-proxy shared-memory writes (barrier init) before later async-proxy accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Untiled bulk copy global -> this CTA's shared memory, completing `bytes` of transaction on
+// `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
                                             int32_t y) {
     asm volatile(

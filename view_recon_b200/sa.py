@@ -30,7 +30,7 @@ EXPORTS = [
     "sa_num_tiles", "sa_max_kept", "sa_tile_pool", "sa_tile_scores", "sa_select_workspace_size",
     "sa_select_topk", "sa_select_topk_noalloc", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
     "sa_dense_attn_fwd",
-    "sa_status_string", "sa_check_device_error", "sa_set_wait_limit_ns",
+    "sa_status_string", "sa_check_device_error", "sa_set_wait_limit_ns", "sa_test_withhold_query_load",
 ]
 
 
@@ -83,6 +83,7 @@ def load(path: str | None = None):
         "sa_status_string": (ctypes.c_char_p, [i32]),
         "sa_check_device_error": (i32, [vp]),
         "sa_set_wait_limit_ns": (i32, [ctypes.c_int64]),
+        "sa_test_withhold_query_load": (i32, [i32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -197,3 +198,7 @@ def sa_check_device_error(stream=None) -> int:
 
 def sa_set_wait_limit_ns(limit_ns: int):
     _check("sa_set_wait_limit_ns", load().sa_set_wait_limit_ns(int(limit_ns)))
+
+
+def sa_test_withhold_query_load(enable: bool):
+    _check("sa_test_withhold_query_load", load().sa_test_withhold_query_load(1 if enable else 0))
