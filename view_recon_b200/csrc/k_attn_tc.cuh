@@ -53,7 +53,7 @@ struct __align__(64) TcArgs {
 // Of every 8 column pairs of a score row, this many take their exponentials on the FMA pipe
 // (exp2_poly2) and the rest on the MUFU (ex2.approx).
 #ifndef SA_EXP2_FMA_PAIRS_PER8
-#define SA_EXP2_FMA_PAIRS_PER8 2
+#define SA_EXP2_FMA_PAIRS_PER8 1
 #endif
 
 namespace tc {
@@ -175,30 +175,6 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
-// Warp-uniform bounded wait for a ping-pong token phase, which also ends as soon as the other
-// slot has finished its items (it then no longer passes the token).
-__device__ __forceinline__ bool wait_token(uint64_t* bar, uint32_t parity, volatile int* other_done,
-                                           volatile int* abort_flag) {
-    bool ok = true;
-    if (!mbar_test(bar, parity)) {
-        const uint64_t t0 = sa_globaltimer();
-        const uint64_t limit = g_sa_wait_limit_ns;
-        for (uint32_t it = 1;; ++it) {
-            if (mbar_test(bar, parity) || *other_done) break;
-            if ((it & 63u) == 0) {
-                if (*abort_flag) { ok = false; break; }
-                if (sa_globaltimer() - t0 > limit) {
-                    sa_flag_error(SA_ERR_TIMEOUT);
-                    *abort_flag = 1;
-                    ok = false;
-                    break;
-                }
-            }
-        }
-    }
-    return __all_sync(0xffffffffu, ok);
-}
-
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred;
     asm volatile(
@@ -224,10 +200,8 @@ struct TcLayout {
     static constexpr int kBars = kKV + NSLOT * STAGES * 2 * tc::kTileBytes;
     // per slot: q_full, kv_full[S], kv_empty[S], s_full, s_free, p_full, pv_done, drain
     static constexpr int kBarsPerSlot = 6 + 2 * STAGES;
-    // ping-pong tokens: tok[x] completes when the other slot has finished a batch of exponentials
-    static constexpr int kTok = kBars + 8 * kBarsPerSlot * NSLOT;
-    static constexpr int kMisc = kTok + 8 * NSLOT;  // tmem base, abort flag, done[NSLOT]
-    static constexpr int kEnd = kMisc + 16 + 4 * NSLOT;
+    static constexpr int kMisc = kBars + 8 * kBarsPerSlot * NSLOT;  // tmem base, abort flag
+    static constexpr int kEnd = kMisc + 16;
     static constexpr uint32_t colS(int x) { return x * 128; }
     static constexpr uint32_t colP(int x) { return NSLOT * 128 + x * 64; }
     static constexpr uint32_t colO(int x) { return NSLOT * 128 + NSLOT * 64 + x * 64; }
@@ -243,8 +217,6 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
-    uint64_t* tok = reinterpret_cast<uint64_t*>(smem + Lay::kTok);             // [NSLOT]
-    volatile int* slot_done = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 16);  // [NSLOT]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool is_softmax = warp >= 4;
@@ -276,8 +248,6 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             mbar_init(&b[3 + 2 * STAGES], 128);    // p_full
             mbar_init(&b[4 + 2 * STAGES], 1);      // pv_done
             mbar_init(&b[5 + 2 * STAGES], 1);      // drain
-            mbar_init(&tok[y], 128);
-            slot_done[y] = 0;
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -407,6 +377,7 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             const int j_cur = j_next;
             if (!a.dense && n + 1 < sl.cnt) j_next = __ldg(sl.list + n + 1);  // one item ahead
             const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
+            if (it.kind < 0 && st == 0) sa_flag_error(SA_ERR_BAD_LIST);  // skipped list entry
             if (!mbar_wait_warp(s_full, n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint32_t sv[128];
@@ -473,14 +444,6 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             if (mx > m_run + 8.0f) m_new = mx;  // lazy max: rescale only on growth beyond 2^8
             const float m_use = m_new == -INFINITY ? 0.0f : m_new;
             const float alpha = ex2_approx(m_run - m_use);  // 0 on the first item
-            // Ping-pong: the two slots take turns on the exponential units, so that one slot's
-            // exponentials overlap the other's TMEM round trips and barrier hand-offs.  Slot 0
-            // runs batch n after slot 1's batch n-1, slot 1 after slot 0's batch n; a slot that
-            // has finished (or given up) no longer holds the other back.
-            if (x == 1 || n > 0) {
-                const uint32_t par = (x == 0 ? (uint32_t)(n - 1) : (uint32_t)n) & 1u;
-                if (!tc::wait_token(&tok[x], par, &slot_done[1 - x], abort_flag)) { ok = false; break; }
-            }
             const float2 mul2 = make_float2(mul, mul);
             const float2 neg2 = make_float2(-m_use, -m_use);
             float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -500,7 +463,6 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                 acc[c & 3] = __fadd2_rn(acc[c & 3], p);
                 pk[c] = pack_bf16x2(p.x, p.y);
             }
-            mbar_arrive(&tok[1 - x]);  // the other slot may start its next batch
             const float2 acc_all = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
             l_run = l_run * alpha + (acc_all.x + acc_all.y);
             m_run = m_new;
@@ -529,7 +491,6 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             tc_fence_before();
             mbar_arrive(p_full);
         }
-        slot_done[x] = 1;  // from here on this slot no longer takes turns
         // ---- epilogue: O / l, LSE, store valid rows
         if (ok && sl.n_items > 0 && mbar_wait_warp(pv_done, (sl.n_items - 1) & 1, abort_flag)) {
             tc_fence_after();
@@ -572,15 +533,6 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             for (int c8 = 0; c8 < 8; ++c8) dst[c8] = make_uint4(0, 0, 0, 0);
             if (a.lse) a.lse[(int64_t)sl.qrow + r] = -INFINITY;
         }
-        // report skipped list entries once per slot
-        if (ok && st == 0 && !a.dense)
-            for (int n = 0; n < sl.cnt; ++n) {
-                const int j = __ldg(sl.list + n);
-                if (j < 0 || j >= a.nt) {
-                    sa_flag_error(SA_ERR_BAD_LIST);
-                    break;
-                }
-            }
     }
 
     tc_fence_before();

@@ -1,28 +1,34 @@
 // Step 3: per-query-tile top-k selection ("SAF3R" abstract: dynamic, input-dependent choice
 // of the most promising interactions; "AVGGT" 2.B.1/2.B.2: own frame and diagonal kept).
 //
-// One 256-thread CTA per score row.  Selection is exact for the order (score descending,
-// tile index ascending).  Scores become order-preserving 32-bit keys (larger float -> larger
-// unsigned key; non-candidates get key 0, candidates at least 1), and the k-th largest key is
-// found MSB first:
-//   1. the row lands in shared memory by one bulk copy; one pass turns it into keys in place
-//      and builds a 4096-bin histogram of the top 12 key bits (sign, exponent, 3 mantissa
-//      bits: a relative resolution of 1/8 octave whatever the scores' scale);
-//   2. the bin holding the k-th largest is found by a block-wide suffix count; one ballot
-//      pass over the row marks every tile above that bin (and the own frame) in a bitmask and
-//      lists the tiles inside it;
-//   3. only the listed tiles are refined, on key bits 19..10 and 9..0, until the remaining
-//      need is a whole bin or the exact threshold key is known;
-//   4. tiles tied at the threshold are admitted in ascending index order by a prefix count
-//      over a tie bitmask, and the bitmask is compacted into ascending indices.
-// Each row is read from memory once; everything after the copy stays on chip.
+// Two kernels with the same result, chosen by row length: short rows (up to
+// SEL_WARP_MAX_NT tiles) take one warp per row, several rows per CTA and no block-wide
+// barrier; long rows take one 256-thread CTA per row (select_topk_block_kernel, below),
+// which keeps enough warps resident when a row fills tens of KB of shared memory.
+// Selection is exact for the order (score descending, tile index ascending).  Scores become order-preserving
+// 32-bit keys (larger float -> larger unsigned key; non-candidates get key 0, candidates at
+// least 1), and the k-th largest key T is found most significant digit first:
+//   1. the row lands in the warp's shared memory by one bulk copy; one pass turns it into
+//      keys in place and builds a 1024-bin histogram of key bits 31..22 (sign, exponent and
+//      one mantissa bit: half-octave bins whatever the scores' scale);
+//   2. a two-step warp search finds the bin holding the k-th largest; the keys inside that
+//      bin are gathered into a short list (or, when the bin is huge, left in the row);
+//   3. the gathered keys alone are refined on bits 21..14, 13..6 and 5..0 until the
+//      remaining need is a whole bin or T itself is known;
+//   4. one ballot pass over the row emits the kept tiles in ascending order: the own frame,
+//      every key above T, and the first `need` keys equal to T in index order.
+// The row is read from memory once; everything after the copy stays in shared memory.
+// The block kernel follows the same plan with a 4096-bin first level over the whole CTA.
 #pragma once
 #include "sa_device.cuh"
 
-#define SEL_THREADS 256
-#define SEL_MAX_NT 32768   // row in shared memory: 128 KB; list indices fit 16 bits
-#define SEL_H1 4096        // first level: key bits 31..20
-#define SEL_H2 1024        // refinement levels: key bits 19..10, then 9..0
+#define SEL_MAX_NT 32768       // row in shared memory: 128 KB
+#define SEL_WARP_MAX_NT 2048   // longest row taken by the warp-per-row kernel
+#define SEL_MAX_WARPS 8
+#define SEL_H1 1024        // first level: key bits 31..22
+#define SEL_H2 256         // refinement digits: bits 21..14, 13..6, 5..0
+#define SEL_LCAP 1024      // boundary-bin keys gathered for refinement
+#define SEL_SMEM_BUDGET (200 * 1024)
 
 struct SelectArgs {
     const float* scores;  // row (local y, local x) at scores + (y * rows + x) * lds
@@ -34,20 +40,241 @@ struct SelectArgs {
     int32_t h0, i0, rows;
 };
 
-// Dynamic shared memory: the row (4 words of slack for alignment), the first-level histogram
-// (later reused as the 16-bit list of boundary tiles), the selection and tie bitmasks.
+// Shared memory of one warp, in words: the row (4 words of slack so that its 16-byte-aligned
+// middle lands 16-byte aligned), the histogram, the gathered keys.
 __host__ __device__ inline size_t select_stage_words(int nt) { return ((size_t)nt + 4 + 3) & ~(size_t)3; }
-__host__ __device__ inline size_t select_list_words(int nt) {
-    const size_t w = ((size_t)nt + 1) / 2;
-    return w > SEL_H1 ? ((w + 3) & ~(size_t)3) : (size_t)SEL_H1;
+__host__ __device__ inline size_t select_warp_words(int nt) { return select_stage_words(nt) + SEL_H1 + SEL_LCAP; }
+// Rows (warps) per CTA for a row length: as many as fit the budget, 1 to SEL_MAX_WARPS.
+__host__ __device__ inline int select_warps(int nt) {
+    const size_t w = (size_t)SEL_SMEM_BUDGET / (4 * select_warp_words(nt));
+    return w < 1 ? 1 : (w > SEL_MAX_WARPS ? SEL_MAX_WARPS : (int)w);
 }
 __host__ __device__ inline size_t select_smem_bytes(int nt) {
-    return 4 * (select_stage_words(nt) + select_list_words(nt) + 2 * (((size_t)nt + 31) / 32));
+    return (size_t)select_warps(nt) * 4 * select_warp_words(nt);
 }
 
 __device__ __forceinline__ uint32_t f32_order_key(float f) {
     const uint32_t b = __float_as_uint(f);
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+struct SelBin {
+    uint32_t bin, above, count, total;  // boundary bin, entries above it, in it, in all bins
+};
+
+// Warp-wide: over NB bins find b with above(b) < want <= above(b) + hist[b], above(b) counting
+// the entries of the bins higher than b, for want = min(want_in, total).  Lane l first sums
+// bins [l*C, l*C+C) (C = NB/32), a suffix scan picks the lane, then that lane's C bins are
+// spread over the warp and scanned the same way.  Meaningful when want >= 1.
+template <int NB>
+__device__ __forceinline__ SelBin sel_find_bin_warp(const uint32_t* hist, uint32_t want_in) {
+    constexpr int C = NB / 32;
+    const int lane = threadIdx.x & 31;
+    uint32_t lsum = 0;
+#pragma unroll
+    for (int u = 0; u < C; u += 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(hist + lane * C + u);
+        lsum += v.x + v.y + v.z + v.w;
+    }
+    uint32_t suf = lsum;  // entries in lanes >= lane
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, suf, off);
+        if (lane + off < 32) suf += y;
+    }
+    SelBin r;
+    r.total = __shfl_sync(0xffffffffu, suf, 0);
+    const uint32_t want = min(want_in, r.total);
+    const uint32_t above_l = suf - lsum;
+    const uint32_t hit = __ballot_sync(0xffffffffu, above_l < want && want <= suf);
+    const int L = hit ? __ffs(hit) - 1 : 0;
+    const uint32_t above_L = __shfl_sync(0xffffffffu, above_l, L);
+    // second step: bin L*C + lane (lanes >= C hold nothing)
+    const uint32_t mine = lane < C ? hist[L * C + lane] : 0u;
+    uint32_t suf2 = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, suf2, off);
+        if (lane + off < 32) suf2 += y;
+    }
+    const uint32_t above2 = above_L + suf2 - mine;
+    const uint32_t hit2 = __ballot_sync(0xffffffffu, lane < C && above2 < want && want <= above2 + mine);
+    const int b = hit2 ? __ffs(hit2) - 1 : 0;
+    r.bin = (uint32_t)(L * C + b);
+    r.above = __shfl_sync(0xffffffffu, above2, b);
+    r.count = __shfl_sync(0xffffffffu, mine, b);
+    return r;
+}
+
+__global__ void __launch_bounds__(32 * SEL_MAX_WARPS) select_topk_warp_kernel(SelectArgs a) {
+    extern __shared__ __align__(16) uint32_t sel_smem[];
+    __shared__ __align__(8) uint64_t bars[SEL_MAX_WARPS];
+    __shared__ int aborts[SEL_MAX_WARPS];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int x = blockIdx.x * nw + warp;  // local row
+    if (x >= a.rows) return;               // no CTA-wide synchronisation follows
+    const int nt = a.nt;
+    uint32_t* stage = sel_smem + (size_t)warp * select_warp_words(nt);
+    uint32_t* hist = stage + select_stage_words(nt);  // [SEL_H1]
+    uint32_t* lkeys = hist + SEL_H1;                  // [SEL_LCAP]
+    uint64_t* bar = &bars[warp];
+    volatile int* abort_flag = &aborts[warp];
+
+    const int h = a.h0 + blockIdx.y, i = a.i0 + x;
+    const float* row = a.scores + ((int64_t)blockIdx.y * a.rows + x) * a.lds;
+    const int f0 = (i / a.tpf) * a.tpf, f1 = f0 + a.tpf;  // own-frame tiles [f0, f1)
+    const int s0 = a.n_sink / a.tile;                      // slots below s0 hold no key row
+
+    // ---- stage the row: one bulk copy for its 16-byte-aligned middle [ha, hb), plain loads
+    // for the (at most 3 + 3) scores at either end; keys[c] = stage[mis + c]
+    const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(row) >> 2) & 3u;
+    const int ha = min(nt, (int)((4u - mis) & 3u));
+    const int n4 = (nt - ha) >> 2;
+    const int hb = ha + 4 * n4;
+    uint32_t* keys = stage + mis;
+    if (lane == 0) {
+        *abort_flag = 0;
+        if (n4 > 0) {
+            mbar_init(bar, 1);
+            fence_barrier_init();
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar, (uint32_t)n4 * 16u);
+            bulk_load(keys + ha, row + ha, (uint32_t)n4 * 16u, bar);
+        }
+    }
+    if (lane < ha) keys[lane] = __float_as_uint(__ldg(row + lane));
+    if (lane >= 16 && lane - 16 < nt - hb) keys[hb + lane - 16] = __float_as_uint(__ldg(row + hb + lane - 16));
+#pragma unroll
+    for (int u = 0; u < SEL_H1 / 128; ++u)
+        reinterpret_cast<uint4*>(hist)[u * 32 + lane] = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
+    if (n4 > 0 && !__all_sync(0xffffffffu, mbar_wait(bar, 0, abort_flag))) return;  // timed out
+
+    // ---- 1. keys in place + first-level histogram
+    auto to_key = [&](int c, uint32_t bits) -> uint32_t {
+        const bool cand = (c < f0 || c >= f1) && (s0 == 0 || c % a.tpf >= s0);
+        if (!cand) return 0u;
+        const uint32_t key = max(f32_order_key(__uint_as_float(bits)), 1u);
+        atomicAdd(&hist[key >> 22], 1u);
+        return key;
+    };
+    if (lane < ha) keys[lane] = to_key(lane, keys[lane]);
+    for (int g = lane; g < n4; g += 32) {
+        uint4* p = reinterpret_cast<uint4*>(keys + ha) + g;
+        uint4 v = *p;
+        const int c = ha + 4 * g;
+        v.x = to_key(c, v.x);
+        v.y = to_key(c + 1, v.y);
+        v.z = to_key(c + 2, v.z);
+        v.w = to_key(c + 3, v.w);
+        *p = v;
+    }
+    if (lane < nt - hb) keys[hb + lane] = to_key(hb + lane, keys[hb + lane]);
+    __syncwarp();
+
+    const uint32_t k_req = (uint32_t)max(a.k, 0);
+    const SelBin b1 = sel_find_bin_warp<SEL_H1>(hist, k_req);
+    const uint32_t ncand = b1.total;
+    const uint32_t kk = min(k_req, ncand);
+    // kept: own frame, key != 0 and ((key >> shift) > prefix, or == prefix and (whole, or
+    // among the first `need` such keys in index order))
+    uint32_t prefix, need = 0;
+    int shift = 0;
+    bool whole;
+    if (kk == 0) {          // none of the candidates
+        prefix = 0xFFFFFFFFu;
+        whole = false;
+    } else if (kk == ncand) {  // all of them
+        prefix = 1u;
+        whole = true;
+    } else {
+        prefix = b1.bin;
+        shift = 22;
+        need = kk - b1.above;
+        whole = need == b1.count;
+    }
+
+    if (!whole && kk > 0) {
+        // ---- 2. gather the keys of the boundary bin (all of them land in the list unless
+        // there are more than SEL_LCAP; then the refinement reads them from the row)
+        uint32_t m = 0;
+        for (int c0 = 0; c0 < nt; c0 += 32) {
+            const int c = c0 + lane;
+            const uint32_t key = c < nt ? keys[c] : 0u;
+            const bool in = key != 0u && (key >> 22) == prefix;
+            const uint32_t bi = __ballot_sync(0xffffffffu, in);
+            const uint32_t pos = m + __popc(bi & ((1u << lane) - 1u));
+            if (in && pos < SEL_LCAP) lkeys[pos] = key;
+            m += __popc(bi);
+        }
+        __syncwarp();
+        const bool from_list = m <= SEL_LCAP;
+        const uint32_t* src = from_list ? lkeys : keys;
+        const int src_n = from_list ? (int)m : nt;
+        // ---- 3. refine on 8, 8 and 6 more bits
+        for (int lvl = 0; lvl < 3 && !whole; ++lvl) {
+            const int width = lvl < 2 ? 8 : 6;
+            const int lo = 14 - 8 * lvl < 0 ? 0 : 14 - 8 * lvl;  // 14, 6, 0
+            const uint32_t digit_mask = (1u << width) - 1u;
+            reinterpret_cast<uint4*>(hist)[lane] = make_uint4(0u, 0u, 0u, 0u);
+            reinterpret_cast<uint4*>(hist)[32 + lane] = make_uint4(0u, 0u, 0u, 0u);
+            __syncwarp();
+            for (int e = lane; e < src_n; e += 32) {
+                const uint32_t key = src[e];
+                if (key != 0u && (key >> (lo + width)) == prefix) atomicAdd(&hist[(key >> lo) & digit_mask], 1u);
+            }
+            __syncwarp();
+            const SelBin r = sel_find_bin_warp<SEL_H2>(hist, need);
+            prefix = (prefix << width) | r.bin;
+            need -= r.above;
+            whole = need == r.count;
+            shift = lo;
+            __syncwarp();
+        }
+    }
+
+    // ---- 4. emit the kept tiles in ascending order
+    int32_t* out = a.kept_idx + ((int64_t)h * nt + i) * a.max_kept;
+    uint32_t pos = 0, tie_before = 0;
+    for (int c0 = 0; c0 < nt; c0 += 32) {
+        const int c = c0 + lane;
+        const uint32_t key = c < nt ? keys[c] : 0u;
+        const uint32_t p = key >> shift;
+        const bool own = c >= f0 && c < f1;
+        const bool above = key != 0u && (p > prefix || (whole && p == prefix));
+        const bool tie = !whole && key != 0u && p == prefix;
+        bool sel = own || above;
+        const uint32_t bt = __ballot_sync(0xffffffffu, tie);
+        if (bt) {
+            sel = sel || (tie && tie_before + __popc(bt & ((1u << lane) - 1u)) < need);
+            tie_before += __popc(bt);
+        }
+        const uint32_t bs = __ballot_sync(0xffffffffu, sel);
+        const uint32_t o = pos + __popc(bs & ((1u << lane) - 1u));
+        if (sel && o < (uint32_t)a.max_kept) out[o] = c;
+        pos += __popc(bs);
+    }
+    uint32_t tot = pos;
+    if (tot > (uint32_t)a.max_kept) {
+        if (lane == 0) sa_flag_error(SA_ERR_INVALID_ARG);
+        tot = a.max_kept;
+    }
+    for (int p = tot + lane; p < a.max_kept; p += 32) out[p] = -1;
+    if (lane == 0) a.kept_cnt[(int64_t)h * nt + i] = (int32_t)tot;
+}
+
+// ----------------------------------------------------------------------------------------------
+// Block-per-row variant (long rows): 256 threads share one staged row.
+#define SEL_BLOCK_THREADS 256
+#define SEL_BLOCK_H1 4096  // first level: key bits 31..20
+#define SEL_BLOCK_H2 1024  // refinement levels: key bits 19..10, then 9..0
+__host__ __device__ inline size_t select_block_stage_words(int nt) { return ((size_t)nt + 4 + 3) & ~(size_t)3; }
+__host__ __device__ inline size_t select_block_list_words(int nt) {
+    const size_t w = ((size_t)nt + 1) / 2;
+    return w > SEL_BLOCK_H1 ? ((w + 3) & ~(size_t)3) : (size_t)SEL_BLOCK_H1;
+}
+__host__ __device__ inline size_t select_block_smem_bytes(int nt) {
+    return 4 * (select_block_stage_words(nt) + select_block_list_words(nt) + 2 * (((size_t)nt + 31) / 32));
 }
 
 // Exclusive scan of one value per thread over the whole block; returns the prefix and
@@ -79,16 +306,16 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
     return before;
 }
 
-struct SelBin {
+struct SelBlockBin {
     uint32_t bin, above, count;  // boundary bin, entries in higher bins, entries in it
 };
 
-// Over BPT * SEL_THREADS bins, find the bin b with above(b) < want <= above(b) + hist[b],
+// Over BPT * SEL_BLOCK_THREADS bins, find the bin b with above(b) < want <= above(b) + hist[b],
 // above(b) counting the entries of the bins higher than b, for want = min(want_in, total).
 // Returns the total; *out is written (and visible to all threads) when want >= 1.
 template <int BPT>
 __device__ __forceinline__ uint32_t sel_find_bin(const uint32_t* hist, uint32_t want_in, uint32_t* scratch,
-                                                 SelBin* out) {
+                                                 SelBlockBin* out) {
     const int tid = threadIdx.x;
     uint32_t bins[BPT], lsum = 0;
 #pragma unroll
@@ -116,19 +343,19 @@ __device__ __forceinline__ uint32_t sel_find_bin(const uint32_t* hist, uint32_t 
     return total;
 }
 
-__global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(SEL_BLOCK_THREADS) select_topk_block_kernel(SelectArgs a) {
     extern __shared__ __align__(16) uint32_t sel_smem[];
     const int nt = a.nt;
     const int nwords = (nt + 31) >> 5;
     uint32_t* stage = sel_smem;
-    uint32_t* hist1 = stage + select_stage_words(nt);   // [SEL_H1], then the list
+    uint32_t* hist1 = stage + select_block_stage_words(nt);   // [SEL_BLOCK_H1], then the list
     uint16_t* lst = reinterpret_cast<uint16_t*>(hist1);
-    uint32_t* selmask = hist1 + select_list_words(nt);  // [nwords]
+    uint32_t* selmask = hist1 + select_block_list_words(nt);  // [nwords]
     uint32_t* eqmask = selmask + nwords;                // [nwords]
-    __shared__ uint32_t hist2[SEL_H2];
+    __shared__ uint32_t hist2[SEL_BLOCK_H2];
     __shared__ uint32_t scratch[32];
     __shared__ __align__(8) uint64_t bar;
-    __shared__ SelBin sb;
+    __shared__ SelBlockBin sb;
     __shared__ uint32_t list_n;
     __shared__ int abort_flag;
 
@@ -160,8 +387,8 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) 
     if (tid < ha) keys[tid] = __float_as_uint(__ldg(row + tid));
     if (tid >= 32 && tid - 32 < nt - hb) keys[hb + tid - 32] = __float_as_uint(__ldg(row + hb + tid - 32));
 #pragma unroll
-    for (int u = 0; u < SEL_H1 / SEL_THREADS; ++u) hist1[u * SEL_THREADS + tid] = 0u;
-    for (int w = tid; w < nwords; w += SEL_THREADS) eqmask[w] = 0u;
+    for (int u = 0; u < SEL_BLOCK_H1 / SEL_BLOCK_THREADS; ++u) hist1[u * SEL_BLOCK_THREADS + tid] = 0u;
+    for (int w = tid; w < nwords; w += SEL_BLOCK_THREADS) eqmask[w] = 0u;
     __syncthreads();
     if (n4 > 0) {
         const bool ok = mbar_wait(&bar, 0, &abort_flag);
@@ -169,7 +396,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) 
     }
 
     // ---- 1. keys in place + first-level histogram
-    for (int c = tid; c < nt; c += SEL_THREADS) {
+    for (int c = tid; c < nt; c += SEL_BLOCK_THREADS) {
         const bool cand = (c < f0 || c >= f1) && (s0 == 0 || c % a.tpf >= s0);
         uint32_t key = 0u;
         if (cand) {
@@ -180,7 +407,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) 
     }
     __syncthreads();
     const uint32_t k_req = (uint32_t)max(a.k, 0);
-    const uint32_t ncand = sel_find_bin<SEL_H1 / SEL_THREADS>(hist1, k_req, scratch, &sb);
+    const uint32_t ncand = sel_find_bin<SEL_BLOCK_H1 / SEL_BLOCK_THREADS>(hist1, k_req, scratch, &sb);
     const uint32_t kk = min(k_req, ncand);
     // selected: own frame, or (key >> shift) > prefix, or == prefix and admitted; with
     // `whole` set every tile at == prefix is admitted
@@ -196,7 +423,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) 
 
     // ---- 2. bitmask of tiles above the boundary bin; list of the tiles inside it (the list
     // overwrites hist1, whose last reads precede the syncs inside sel_find_bin)
-    for (int wd = warp; wd < nwords; wd += SEL_THREADS / 32) {
+    for (int wd = warp; wd < nwords; wd += SEL_BLOCK_THREADS / 32) {
         const int c = wd * 32 + lane;
         const uint32_t key = c < nt ? keys[c] : 0u;
         const bool own = c >= f0 && c < f1;
@@ -227,14 +454,14 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) 
         const uint32_t m = list_n;
         for (int lvl = 0; lvl < 2 && !whole; ++lvl) {
             const int sh = 10 - 10 * lvl;
-            for (int b = tid; b < SEL_H2; b += SEL_THREADS) hist2[b] = 0u;
+            for (int b = tid; b < SEL_BLOCK_H2; b += SEL_BLOCK_THREADS) hist2[b] = 0u;
             __syncthreads();
-            for (uint32_t e = tid; e < m; e += SEL_THREADS) {
+            for (uint32_t e = tid; e < m; e += SEL_BLOCK_THREADS) {
                 const uint32_t key = keys[lst[e]];
-                if ((key >> (sh + 10)) == prefix) atomicAdd(&hist2[(key >> sh) & (SEL_H2 - 1)], 1u);
+                if ((key >> (sh + 10)) == prefix) atomicAdd(&hist2[(key >> sh) & (SEL_BLOCK_H2 - 1)], 1u);
             }
             __syncthreads();
-            sel_find_bin<SEL_H2 / SEL_THREADS>(hist2, need, scratch, &sb);
+            sel_find_bin<SEL_BLOCK_H2 / SEL_BLOCK_THREADS>(hist2, need, scratch, &sb);
             prefix = (prefix << 10) | sb.bin;
             need -= sb.above;
             whole = need == sb.count;
@@ -243,7 +470,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) 
         }
         // admit the listed tiles above the threshold (and at it, when all of them are taken);
         // mark ties otherwise
-        for (uint32_t e = tid; e < m; e += SEL_THREADS) {
+        for (uint32_t e = tid; e < m; e += SEL_BLOCK_THREADS) {
             const int c = lst[e];
             const uint32_t p = keys[c] >> shift;
             if (p > prefix || (whole && p == prefix))
@@ -255,7 +482,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) 
     }
 
     // ---- 4. ties in index order, then compaction; thread t owns words [w0, w1)
-    const int wpt = (nwords + SEL_THREADS - 1) / SEL_THREADS;  // <= 4
+    const int wpt = (nwords + SEL_BLOCK_THREADS - 1) / SEL_BLOCK_THREADS;  // <= 4
     const int w0 = min(nwords, tid * wpt), w1 = min(nwords, w0 + wpt);
     uint32_t tot;
     if (mode == 2 && !whole) {  // shift == 0 here: the tied tiles share the exact threshold key
@@ -293,6 +520,6 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk_kernel(SelectArgs a) 
         if (tid == 0) sa_flag_error(SA_ERR_INVALID_ARG);
         tot = a.max_kept;
     }
-    for (int p = tot + tid; p < a.max_kept; p += SEL_THREADS) out[p] = -1;
+    for (int p = tot + tid; p < a.max_kept; p += SEL_BLOCK_THREADS) out[p] = -1;
     if (tid == 0) a.kept_cnt[(int64_t)h * nt + i] = (int32_t)tot;
 }

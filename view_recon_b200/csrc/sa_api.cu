@@ -100,8 +100,10 @@ sa_status ensure_attributes() {
                                200 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                200 * 1024) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)select_smem_bytes(SEL_MAX_NT)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SEL_SMEM_BUDGET) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_topk_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)select_block_smem_bytes(SEL_MAX_NT)) == cudaSuccess;
     // The tensor-core kernel moves registers between its warpgroups (setmaxnreg); that is only
     // satisfiable if the block is launched with at least the registers the split hands out.
     cudaFuncAttributes fa;
@@ -502,6 +504,19 @@ size_t sa_select_workspace_size(const sa_shape* shape, int32_t streamed) {
     return select_rows_per_block(g) * (size_t)g.nt * 4;
 }
 
+// Short rows: one warp per row, as many rows per CTA as fit in shared memory; long rows:
+// one 256-thread CTA per row.
+static void launch_select(const SelectArgs& a, unsigned gy, cudaStream_t stream) {
+    if (a.nt <= SEL_WARP_MAX_NT) {
+        const int w = select_warps(a.nt);
+        const unsigned gx = (unsigned)((a.rows + w - 1) / w);
+        select_topk_warp_kernel<<<dim3(gx, gy), 32 * w, select_smem_bytes(a.nt), stream>>>(a);
+    } else {
+        select_topk_block_kernel<<<dim3((unsigned)a.rows, gy), SEL_BLOCK_THREADS, select_block_smem_bytes(a.nt),
+                                   stream>>>(a);
+    }
+}
+
 sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, const float* q_pool,
                          const float* k_pool, int32_t k, int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
                          void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream) {
@@ -530,14 +545,13 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, con
     a.n_sink = (int32_t)g.n_sink;
     a.k = k;
     a.max_kept = max_kept;
-    const size_t smem = select_smem_bytes((int)g.nt);
     if (scores_or_null) {
         a.scores = scores_or_null;
         a.lds = g.nt;
         a.h0 = 0;
         a.i0 = 0;
         a.rows = (int32_t)g.nt;
-        select_topk_kernel<<<dim3((unsigned)g.nt, (unsigned)g.bh), SEL_THREADS, smem, stream>>>(a);
+        launch_select(a, (unsigned)g.bh, stream);
         return launch_status();
     }
     // streamed: score one L2-resident block of rows at a time, then select from it
@@ -563,7 +577,7 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, con
             a.h0 = (int32_t)h;
             a.i0 = (int32_t)i0;
             a.rows = (int32_t)rows;
-            select_topk_kernel<<<dim3((unsigned)rows, 1), SEL_THREADS, smem, stream>>>(a);
+            launch_select(a, 1u, stream);
             if ((st = launch_status()) != SA_OK) return st;
         }
     }
@@ -594,7 +608,6 @@ sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, con
     a.n_sink = (int32_t)g.n_sink;
     a.k = k;
     a.max_kept = max_kept;
-    const size_t smem = select_smem_bytes((int)g.nt);
     for (int64_t h = 0; h < g.bh; ++h) {
         for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
             const int64_t rows = std::min<int64_t>(R, g.nt - i0);
@@ -615,7 +628,7 @@ sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, con
             a.h0 = (int32_t)h;
             a.i0 = (int32_t)i0;
             a.rows = (int32_t)rows;
-            select_topk_kernel<<<dim3((unsigned)rows, 1), SEL_THREADS, smem, stream>>>(a);
+            launch_select(a, 1u, stream);
             if ((st = launch_status()) != SA_OK) return st;
         }
     }
