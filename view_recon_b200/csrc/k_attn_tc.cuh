@@ -53,7 +53,7 @@ struct __align__(64) TcArgs {
 // Of every 8 column pairs of a score row, this many take their exponentials on the FMA pipe
 // (exp2_poly2) and the rest on the MUFU (ex2.approx).
 #ifndef SA_EXP2_FMA_PAIRS_PER8
-#define SA_EXP2_FMA_PAIRS_PER8 1
+#define SA_EXP2_FMA_PAIRS_PER8 2
 #endif
 
 namespace tc {
@@ -371,11 +371,10 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
         const uint32_t tO = tmem + Lay::colO(x) + lane_off;
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
-        int j_next = (!a.dense && sl.cnt > 0) ? __ldg(sl.list) : 0;  // list entry of the next item
         int lm_ptr = 0;                                              // landmark chunks: list cursor
         for (int n = 0; n < sl.n_items; ++n) {
-            const int j_cur = j_next;
-            if (!a.dense && n + 1 < sl.cnt) j_next = __ldg(sl.list + n + 1);  // one item ahead
+            const int j_cur = (!a.dense && n < sl.cnt) ? __ldg(sl.list + n) : 0;  // (a prefetch one item ahead
+            // measured slower: it lengthens register live ranges in this loop)
             const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
             if (it.kind < 0 && st == 0) sa_flag_error(SA_ERR_BAD_LIST);  // skipped list entry
             if (!mbar_wait_warp(s_full, n & 1, abort_flag)) { ok = false; break; }
