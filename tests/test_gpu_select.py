@@ -46,6 +46,7 @@ def score_rows(bh, nt, seed):
     (200, 1374, 128, 5, 130, 2),    # 2200 tiles: block-per-row kernel
     (190, 1374, 128, 256, 40, 1),   # block kernel, two whole sink slots per frame excluded
     (30, 1374, 128, 256, 0, 1),     # k = 0: own frame only
+    (40, 700, 128, 256, 9, 2),      # warp kernel with two whole sink slots per frame
 ])
 def test_selection_exact_on_stress_rows(frames, tokens, tile, n_sink, k, bh):
     import torch

@@ -150,10 +150,10 @@ __global__ void __launch_bounds__(32 * SEL_MAX_WARPS) select_topk_warp_kernel(Se
     __syncwarp();
     if (n4 > 0 && !__all_sync(0xffffffffu, mbar_wait(bar, 0, abort_flag))) return;  // timed out
 
-    // ---- 1. keys in place + first-level histogram
+    // ---- 1. keys in place + first-level histogram (every tile outside the own frame counts
+    // here; tiles of whole sink slots are taken out afterwards, without a division per tile)
     auto to_key = [&](int c, uint32_t bits) -> uint32_t {
-        const bool cand = (c < f0 || c >= f1) && (s0 == 0 || c % a.tpf >= s0);
-        if (!cand) return 0u;
+        if (c >= f0 && c < f1) return 0u;
         const uint32_t key = max(f32_order_key(__uint_as_float(bits)), 1u);
         atomicAdd(&hist[key >> 22], 1u);
         return key;
@@ -171,6 +171,17 @@ __global__ void __launch_bounds__(32 * SEL_MAX_WARPS) select_topk_warp_kernel(Se
     }
     if (lane < nt - hb) keys[hb + lane] = to_key(hb + lane, keys[hb + lane]);
     __syncwarp();
+    if (s0 > 0) {  // slots below s0 hold sink rows only: not candidates
+        for (int e = lane; e < (nt / a.tpf) * s0; e += 32) {
+            const int fr = e / s0, c = fr * a.tpf + (e - fr * s0);
+            const uint32_t key = keys[c];
+            if (key != 0u) {
+                atomicSub(&hist[key >> 22], 1u);
+                keys[c] = 0u;
+            }
+        }
+        __syncwarp();
+    }
 
     const uint32_t k_req = (uint32_t)max(a.k, 0);
     const SelBin b1 = sel_find_bin_warp<SEL_H1>(hist, k_req);
@@ -395,17 +406,27 @@ __global__ void __launch_bounds__(SEL_BLOCK_THREADS) select_topk_block_kernel(Se
         if (__syncthreads_or(!ok)) return;  // timed out: the error word says so
     }
 
-    // ---- 1. keys in place + first-level histogram
+    // ---- 1. keys in place + first-level histogram (sink slots taken out afterwards)
     for (int c = tid; c < nt; c += SEL_BLOCK_THREADS) {
-        const bool cand = (c < f0 || c >= f1) && (s0 == 0 || c % a.tpf >= s0);
         uint32_t key = 0u;
-        if (cand) {
+        if (c < f0 || c >= f1) {
             key = max(f32_order_key(__uint_as_float(keys[c])), 1u);
             atomicAdd(&hist1[key >> 20], 1u);
         }
         keys[c] = key;
     }
     __syncthreads();
+    if (s0 > 0) {  // slots below s0 hold sink rows only: not candidates
+        for (int e = tid; e < (nt / a.tpf) * s0; e += SEL_BLOCK_THREADS) {
+            const int fr = e / s0, c = fr * a.tpf + (e - fr * s0);
+            const uint32_t key = keys[c];
+            if (key != 0u) {
+                atomicSub(&hist1[key >> 20], 1u);
+                keys[c] = 0u;
+            }
+        }
+        __syncthreads();
+    }
     const uint32_t k_req = (uint32_t)max(a.k, 0);
     const uint32_t ncand = sel_find_bin<SEL_BLOCK_H1 / SEL_BLOCK_THREADS>(hist1, k_req, scratch, &sb);
     const uint32_t kk = min(k_req, ncand);
