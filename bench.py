@@ -2,6 +2,7 @@
 """Benchmark: one sparse global-attention layer call (pool -> score -> select -> attend) per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+                    [--shard replicas|heads]
 
 Prints ONE JSON line (rank 0).  `value` is whole-job tokens/s on the device with inputs
 resident in HBM (CUDA events on the launching stream, L2 flushed before every step, max over
@@ -9,10 +10,12 @@ ranks); `e2e` is the same metric through the public API with host-resident pinne
 host->device copies of Q/K/V and the device->host read of O inside every timed step.
 `roofline` reports the block-sparse attention kernel against the measured bf16 peak, and
 `cpu_baseline` the fp64 CPU oracle on a bounded sample of the same workload.
-With N > 1 (torchrun) every rank runs its own independent layer call (a different seed:
-heads/batches are independent problems), so per-GPU work is fixed ("scaling": "weak") and
+With N > 1 (torchrun) every rank runs its own independent layer call by default (a different
+seed: heads/batches are independent problems), so per-GPU work is fixed ("scaling": "weak");
+with --shard heads the ranks split ONE layer call by heads ("scaling": "strong").  Either way
 no collective touches the data path; a barrier and a max-reduction of the timings are the
-only cross-rank operations.
+only cross-rank operations.  The overlapped host pipeline (`e2e`) copies every call's inputs
+in and its output out inside the timed region.
 """
 from __future__ import annotations
 
@@ -52,6 +55,25 @@ def rank_env():
 def rank_seed(base_seed: int, rank: int) -> int:
     """Each rank draws an independent problem (weak scaling over independent layer calls)."""
     return base_seed + 1000 * rank
+
+
+def shard_plan(mode: str, heads: int, world: int, rank: int, base_seed: int):
+    """How one rank's work relates to the job.
+
+    mode "replicas": every rank runs its own independent layer call (its own seed), so the job
+    is `world` layer calls and per-GPU work is fixed ("weak" scaling).
+    mode "heads": the ranks share one layer call; rank r takes heads [r*H/world, (r+1)*H/world)
+    of the same draw.  Heads are independent problems end to end, so no data moves between
+    ranks ("strong" scaling).
+    Returns (heads on this rank, first head, seed, layer calls this rank contributes).
+    """
+    if mode == "heads" and world > 1:
+        if heads % world:
+            raise ValueError("--shard heads needs the head count (%d) divisible by the GPU count (%d)"
+                             % (heads, world))
+        hl = heads // world
+        return hl, rank * hl, base_seed, 1.0 / world
+    return heads, 0, rank_seed(base_seed, rank), 1.0
 
 
 def dist_max(value: float, device=None) -> float:
@@ -246,7 +268,7 @@ def run_ours(args, w):
 
     import synth
     from view_recon_b200 import sa
-    from view_recon_b200.pipeline import SparseGlobalAttention
+    from view_recon_b200.pipeline import HostPipeline, SparseGlobalAttention
 
     rank, world, local = rank_env()
     if world > 1:
@@ -257,8 +279,10 @@ def run_ours(args, w):
     torch.cuda.set_device(dev)
     sa.load()
 
-    seed = rank_seed(w.seed, rank)
-    host = synth.generate(w, seed=seed)
+    w_job = w
+    heads_local, head0, seed, calls_here = shard_plan(args.shard, w.heads, world, rank, w.seed)
+    w = w.scaled(heads=heads_local)
+    host = synth.generate(w, seed=seed, head0=head0)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def pinned(a):
@@ -332,28 +356,25 @@ def run_ours(args, w):
     torch.cuda.synchronize(dev)
     dense_ms = float(np.mean([a.elapsed_time(b) for a, b in d_ms]))
 
-    # end to end through the public API from pinned host buffers
+    # end to end through the public API from pinned host buffers: every call copies its Q/K/V in
+    # and its O out; HostPipeline overlaps call i's kernels with the copies of calls i+1 and i-1
     ho = torch.empty((w.heads, w.L, w.head_dim), dtype=tdt).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
-
-    def e2e_step():
-        qd = hq.to(dev, non_blocking=True)
-        kd = hk.to(dev, non_blocking=True)
-        vd = hv.to(dev, non_blocking=True)
-        o, _ = layer.forward(qd, kd, vd)
-        ho.copy_(o, non_blocking=True)
-
+    pipe = HostPipeline(lambda: SparseGlobalAttention(w.heads, w.frames, w.tokens, w.k, w.tile, w.n_sink, w.dtype,
+                                                      w.landmark, w.streamed, w.head_dim, device=dev))
     for _ in range(2):
-        e2e_step()
+        pipe.submit(hq, hk, hv, ho)
+    pipe.synchronize()
     torch.cuda.synchronize(dev)
     dist_barrier(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(pipe.s_in)
     for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+        pipe.submit(hq, hk, hv, ho)
+    e1.record(pipe.s_out)
     torch.cuda.synchronize(dev)
     e2e_ms = dist_max(e0.elapsed_time(e1), dev)
+    del pipe
     elem = 2 if w.dtype == "bf16" else 4
     h2d = 3 * w.heads * w.L * w.head_dim * elem
     d2h = w.heads * w.L * w.head_dim * elem
@@ -362,7 +383,8 @@ def run_ours(args, w):
     achieved = flops / (ms_attn / 1e3) / 1e12
     traffic = profiled_traffic(w.name)
     per_step = layer.launches_per_call()
-    value = whole_job_rate(w.L, world, args.steps, max_total_ms)
+    value = whole_job_rate(w.L * calls_here, world, args.steps, max_total_ms)
+    sharded = args.shard == "heads" and world > 1
     line = {
         "metric": METRIC,
         "value": value,
@@ -372,15 +394,16 @@ def run_ours(args, w):
         "warmup": args.warmup,
         "ms_per_step": max_total_ms / args.steps,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic latent-point Q/K/V (seeded; no dataset or weights)",
-        "config": {"workload": w.name, "frames": w.frames, "tokens_per_frame": w.tokens, "heads": w.heads,
+        "config": {"workload": w_job.name, "frames": w.frames, "tokens_per_frame": w.tokens, "heads": w_job.heads,
                    "head_dim": w.head_dim, "tile": w.tile, "n_sink": w.n_sink, "k": w.k,
                    "kept_tiles_per_query_tile": layer.max_kept, "tile_sparsity": round(w.sparsity, 4),
                    "landmark": w.landmark, "streamed_select": w.streamed, "l2": "flushed before every step",
-                   "parallelism": "independent layer call per GPU" if world > 1 else "single GPU"},
+                   "parallelism": ("%d heads per GPU, one layer call over %d GPUs" % (w.heads, world)) if sharded
+                   else ("independent layer call per GPU" if world > 1 else "single GPU")},
         "stages_ms": {"pool": ms_pool, "score": ms_score, "select": ms_select, "attn": ms_attn},
         "attn_tflops_algorithmic": achieved,
         "attn_tflops_kept_tiles": tile_flops / (ms_attn / 1e3) / 1e12,
@@ -394,7 +417,7 @@ def run_ours(args, w):
                      "peak_source": "%s bf16 burst" % peak_src,
                      "traffic": (traffic if traffic is None else traffic),
                      "algorithmic_flops_per_launch": flops},
-        "e2e": {"value": whole_job_rate(w.L, world, e2e_steps, e2e_ms), "unit": UNIT,
+        "e2e": {"value": whole_job_rate(w.L * calls_here, world, e2e_steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": per_step * args.steps,
         "clocks": clk,
@@ -406,6 +429,122 @@ def run_ours(args, w):
     if rank == 0:
         print(json.dumps(line), flush=True)
     del layer
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------ SGA arm
+
+def run_sga(args, w):
+    """--sga S: the AVGGT subsampled global attention layer (stride S x S on the 37 x 37 patch grid
+    of every frame) on the workload's shape, through the same timing contract."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from view_recon_b200 import sa
+    from view_recon_b200.pipeline import HostPipeline, SubsampledGlobalAttention
+
+    rank, world, local = rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    sa.load()
+    grid = int(round((w.tokens - w.n_sink) ** 0.5))
+    if grid * grid + w.n_sink != w.tokens:
+        raise SystemExit("--sga needs tokens = n_sink + g * g")
+    stride = int(args.sga)
+    w_job = w
+    heads_local, head0, seed, calls_here = shard_plan(args.shard, w.heads, world, rank, w.seed)
+    w = w.scaled(heads=heads_local)
+    host = synth.generate(w, seed=seed, head0=head0)
+
+    def pinned(a):
+        return torch.from_numpy(a).view(torch.bfloat16).pin_memory()
+
+    hq, hk, hv = pinned(host["q"]), pinned(host["k"]), pinned(host["v"])
+    q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
+    make = lambda: SubsampledGlobalAttention(w.heads, w.frames, w.tokens, (grid, grid), (stride, stride),  # noqa: E731
+                                             w.n_sink, w.dtype, w.head_dim, device=dev)
+    layer = make()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer.forward(q, k, v)
+    torch.cuda.synchronize(dev)
+    if sa.sa_check_device_error() != 0:
+        raise RuntimeError("device error after warm-up")
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    dist_barrier(dev)
+    torch.cuda.synchronize(dev)
+    evs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        layer.forward(q, k, v)
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    dist_barrier(dev)
+    clk = clocks.stop()
+    total_ms = float(sum(a.elapsed_time(b) for a, b in evs))
+    max_total_ms = dist_max(total_ms, dev)
+    ms = total_ms / args.steps
+    # end to end from pinned host buffers
+    ho = torch.empty_like(hq).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    pipe = HostPipeline(make)
+    for _ in range(2):
+        pipe.submit(hq, hk, hv, ho)
+    pipe.synchronize()
+    dist_barrier(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(pipe.s_in)
+    for _ in range(e2e_steps):
+        pipe.submit(hq, hk, hv, ho)
+    e1.record(pipe.s_out)
+    torch.cuda.synchronize(dev)
+    e2e_ms = dist_max(e0.elapsed_time(e1), dev)
+    del pipe
+    # algorithmic work: every query row over the compacted keys, its diagonal and the mean pair
+    flops = 4.0 * w.head_dim * w.heads * float(w.L) * float(layer.kept_keys + 2)
+    peaks, peak_src = measured_peaks()
+    achieved = flops / (ms / 1e3) / 1e12
+    elem = 2
+    sharded = args.shard == "heads" and world > 1
+    line = {
+        "metric": METRIC, "value": whole_job_rate(w.L * calls_here, world, args.steps, max_total_ms),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": max_total_ms / args.steps, "higher_is_better": True,
+        "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic latent-point Q/K/V (seeded; no dataset or weights)",
+        "config": {"workload": "%s_sga%d" % (w_job.name, stride), "frames": w.frames, "tokens_per_frame": w.tokens,
+                   "heads": w_job.heads, "head_dim": w.head_dim, "grid": [grid, grid], "stride": [stride, stride],
+                   "n_special": w.n_sink, "kept_keys_per_head": layer.kept_keys,
+                   "l2": "flushed before every step",
+                   "parallelism": ("%d heads per GPU, one layer call over %d GPUs" % (w.heads, world)) if sharded
+                   else ("independent layer call per GPU" if world > 1 else "single GPU")},
+        "stages_ms": {"sga": ms},
+        "attn_tflops_algorithmic": achieved,
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (dense over the kept keys)",
+                     "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "peak_source": "%s bf16 burst" % peak_src,
+                     "traffic": None, "algorithmic_flops_per_launch": flops},
+        "e2e": {"value": whole_job_rate(w.L * calls_here, world, e2e_steps, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": 3 * w.heads * w.L * w.head_dim * elem,
+                "d2h_bytes_per_step": w.heads * w.L * w.head_dim * elem},
+        "gpu_launches": 5 * args.steps,  # gather, sums, V^T tiles, attention, combine
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 
@@ -449,6 +588,10 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sga", type=int, default=0, metavar="STRIDE",
+                    help="time the AVGGT subsampled global attention layer (stride x stride grid) instead")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="with N > 1: independent layer call per GPU, or one layer call split by heads")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
     args = ap.parse_args(argv)
@@ -457,6 +600,8 @@ def main(argv=None):
     w = BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.sga:
+        run_sga(args, w)
     else:
         run_ours(args, w)
 

@@ -147,6 +147,27 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null,
                          void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream);
 
 /*
+ * sa_select_topk with a budget per head (SAF3R abstract: attention sparsity differs across
+ * heads, and the budgets come from offline head profiling and online adaptation; neither the
+ * profile nor the adaptation rule is part of this library - the caller supplies the budgets).
+ *   k_per_head  int32 [bh], DEVICE memory, 4-byte aligned: head h keeps the k_per_head[h]
+ *               best candidate tiles (all of them when the budget reaches their number, i.e.
+ *               a dense head; 0 keeps the own frame only).  Read on the device when the
+ *               kernels run, so the budgets may be computed on the GPU in the same stream.
+ *   k_max       an upper bound on every entry, >= 0; max_kept >= sa_max_kept(shape, k_max).
+ *               An entry below 0 or above k_max is clamped into [0, k_max] and reported as
+ *               SA_ERR_INVALID_ARG by sa_check_device_error.
+ * Everything else, outputs included, is as for sa_select_topk; kept_cnt varies by head and
+ * sa_sparse_attn_fwd consumes the lists unchanged.  Returns SA_ERR_INVALID_ARG for a NULL or
+ * misaligned k_per_head or k_max < 0, before any launch.
+ */
+sa_status sa_select_topk_per_head(const sa_shape* shape, const float* scores_or_null,
+                                  const float* q_pool, const float* k_pool,
+                                  const int32_t* k_per_head, int32_t k_max,
+                                  int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
+                                  void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream);
+
+/*
  * sa_select_topk in streamed mode without any caller-provided memory.  No passage of the
  * pages corresponds to this call; it exists for callers that cannot allocate device memory
  * where this step runs - for instance plugin code inside a host framework that owns the
@@ -223,6 +244,30 @@ sa_status sa_check_device_error(sa_stream_t stream);
  * device (default 2e9, i.e. 2 s; must be > 0).  A wait that runs out ends its kernel early
  * with SA_ERR_TIMEOUT recorded; outputs of that launch are then undefined. */
 sa_status sa_set_wait_limit_ns(int64_t limit_ns);
+
+/*
+ * Subsampled global attention ("AVGGT: Rethinking Global Attention for Accelerating VGGT",
+ * technical summary 2.B.2, SGA), an alternative to steps 1-4 for the later global layers.
+ * Every frame is shape->n_sink special tokens followed by a grid_h x grid_w patch grid in
+ * row-major order (shape->tokens == n_sink + grid_h * grid_w).  Keys and values are kept for
+ * the special tokens of every frame and for the patches at (r, c) with r a multiple of s_h
+ * and c a multiple of s_w (one per s_h x s_w window); every query is kept.  Query t attends to
+ *   - every kept key of every frame,
+ *   - its own key (the diagonal), when its token is not among the kept ones,
+ *   - one mean key/value pair standing for the other discarded tokens of all frames
+ *     (mean K, mean V over them; logit scale * q.k_mean + ln(their count)),
+ * with softmax_scale as for sa_sparse_attn_fwd.  Output O [bh][S*N][64] and, when lse_or_null
+ * is given, the natural-log LSE [bh][S*N] of that softmax.
+ * Built for bf16, head_dim 64 and tile 128 (the tensor-core path; SA_ERR_UNSUPPORTED else).
+ * workspace: >= sa_sga_workspace_size(...) bytes, 16-byte aligned (the compacted K/V
+ * sequence, fp32 sums of the discarded rows, an LSE scratch and the attention's V^T tiles).
+ * SA_ERR_INVALID_ARG for a grid that does not match shape->tokens, strides < 1, NULL or
+ * misaligned pointers; all checked on the host before any launch.
+ */
+size_t sa_sga_workspace_size(const sa_shape* shape, int32_t grid_h, int32_t grid_w, int32_t s_h, int32_t s_w);
+sa_status sa_sga_fwd(const sa_shape* shape, int32_t grid_h, int32_t grid_w, int32_t s_h, int32_t s_w,
+                     const void* q, const void* k, const void* v, void* workspace, size_t workspace_bytes,
+                     void* o, float* lse_or_null, sa_stream_t stream);
 
 /* Test facility for the failure path (not for production use): while enable != 0, later
  * launches of the tensor-core attention kernel (bf16, tile 128) on the current device never

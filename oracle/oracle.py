@@ -187,6 +187,16 @@ def select(g: Geometry, s: np.ndarray, k: int):
     return [[select_row(g, s[h, i], i, k) for i in range(g.nt)] for h in range(bh)]
 
 
+def select_per_head(g: Geometry, s: np.ndarray, k_per_head):
+    """kept[h][i] when head h keeps its own budget k_per_head[h] of candidate tiles.
+
+    Attention sparsity differs from head to head, and budgets are set per head from offline
+    profiling and online adaptation ("SAF3R" abstract).  The selection rule of each head is
+    the single-budget rule; a budget at or above the candidate count makes that head dense.
+    """
+    return [[select_row(g, s[h, i], i, int(k_per_head[h])) for i in range(g.nt)] for h in range(s.shape[0])]
+
+
 def max_kept(g: Geometry, k: int) -> int:
     """Length of every kept list: own-frame tiles plus min(k, candidates)."""
     n_cand = (g.frames - 1) * sum(1 for slot in range(g.tpf) if g.key_count(slot) > 0)
@@ -288,6 +298,69 @@ def attend_bruteforce(g: Geometry, q, k, v, kept, scale: float, landmark: bool =
             bias = bias[:, :L]
         logits = scale * (q[h] @ keys.T) + bias
         O[h], LSE[h] = _softmax_rows(logits, vals)
+    return O, LSE
+
+
+# ----------------------------------------------------------------------------- subsampled global attention
+
+def sga_kept(frames: int, tokens: int, n_special: int, grid_h: int, grid_w: int, s_h: int, s_w: int):
+    """Boolean [S*N]: the key/value tokens a subsampled global attention layer keeps.
+
+    Every frame is n_special special tokens followed by a grid_h x grid_w patch grid in
+    row-major order.  Kept: all special tokens, and the patch at (r, c) when r is a multiple of
+    s_h and c a multiple of s_w - one token per s_h x s_w window of the 2-D grid ("AVGGT",
+    technical summary 2.B.2, "Estrategia de Grade": keys and values subsampled uniformly on a
+    2-D grid; special tokens preserved).
+    """
+    if n_special + grid_h * grid_w != tokens:
+        raise ValueError("tokens must be n_special + grid_h * grid_w")
+    per = np.zeros((tokens,), bool)
+    per[:n_special] = True
+    r = np.arange(grid_h)[:, None]
+    c = np.arange(grid_w)[None, :]
+    per[n_special:] = ((r % s_h == 0) & (c % s_w == 0)).reshape(-1)
+    return np.tile(per, frames)
+
+
+def sga(q, k, v, frames: int, tokens: int, n_special: int, grid_h: int, grid_w: int, s_h: int, s_w: int,
+        scale: float):
+    """Subsampled global attention ("AVGGT", technical summary 2.B.2, SGA).
+
+    Every query attends to the kept tokens (sga_kept), to its own key (the diagonal is
+    preserved explicitly), and to one extra key/value pair standing for the discarded columns:
+    the mean key and mean value of the discarded tokens of all frames - for a query whose own
+    token is discarded, all of them except itself, since its column is kept as the diagonal -
+    with a logit bias of ln(count), so that the pair weighs as the columns it replaces (the
+    aggregated response of the discarded columns is kept).  Returns (O [bh][L][d], LSE [bh][L]).
+    """
+    bh, L, _ = q.shape
+    kept = sga_kept(frames, tokens, n_special, grid_h, grid_w, s_h, s_w)
+    disc = np.nonzero(~kept)[0]
+    kidx = np.nonzero(kept)[0]
+    n_d = len(disc)
+    O = np.zeros((bh, L, v.shape[2]))
+    LSE = np.zeros((bh, L))
+    for h in range(bh):
+        k_sum = k[h, disc].sum(axis=0)
+        v_sum = v[h, disc].sum(axis=0)
+        for t in range(L):
+            own_disc = not kept[t]
+            keys = [k[h, kidx]]
+            vals = [v[h, kidx]]
+            logits = [scale * (k[h, kidx] @ q[h, t])]
+            if own_disc:  # the diagonal
+                keys.append(k[h, t][None])
+                vals.append(v[h, t][None])
+                logits.append(np.array([scale * (k[h, t] @ q[h, t])]))
+            c = n_d - (1 if own_disc else 0)
+            if c > 0:  # the mean pair of the other discarded columns
+                kb = (k_sum - (k[h, t] if own_disc else 0.0)) / c
+                vb = (v_sum - (v[h, t] if own_disc else 0.0)) / c
+                vals.append(vb[None])
+                logits.append(np.array([scale * (kb @ q[h, t]) + math.log(c)]))
+            lg = np.concatenate(logits)[None, :]
+            o, lse = _softmax_rows(lg, np.concatenate(vals, axis=0))
+            O[h, t], LSE[h, t] = o[0], lse[0]
     return O, LSE
 
 

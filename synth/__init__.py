@@ -35,6 +35,7 @@ class _Cfg(ctypes.Structure):
         ("seed", ctypes.c_uint64),
         ("out_bf16", ctypes.c_int32),
         ("n_threads", ctypes.c_int32),
+        ("head0", ctypes.c_int32),
     ]
 
 
@@ -68,13 +69,14 @@ def default_threads() -> int:
 
 
 def generate(w: Workload, seed: int | None = None, heads: int | None = None,
-             threads: int | None = None, dtype: str | None = None):
+             threads: int | None = None, dtype: str | None = None, head0: int = 0):
     """Return dict(q, k, v, point) as numpy arrays.
 
     q, k, v have shape [heads][S*N][d]; bf16 workloads come back as uint16
     bit patterns, f32 workloads as float32.  `point` is the int32 point id of
     every token (-1 = untied).  `heads` overrides the head count (heads are
-    independent draws, so the first h heads of a larger draw are identical).
+    independent draws, so the first h heads of a larger draw are identical); `head0`
+    draws heads head0 .. head0 + heads - 1 of that larger draw instead (a head shard).
     """
     lib = _load()
     dt = dtype or w.dtype
@@ -82,7 +84,7 @@ def generate(w: Workload, seed: int | None = None, heads: int | None = None,
     cfg = _Cfg(bh, w.frames, w.tokens, w.head_dim, w.n_sink, w.n_points, w.window,
                float(w.p_assign), A_LAT, A_NOISE, SINK_K_SCALE,
                int(w.seed if seed is None else seed), 1 if dt == "bf16" else 0,
-               int(threads or default_threads()))
+               int(threads or default_threads()), int(head0))
     shape = (bh, w.L, w.head_dim)
     npdt = np.uint16 if dt == "bf16" else np.float32
     q = np.empty(shape, npdt)
@@ -96,7 +98,7 @@ def generate(w: Workload, seed: int | None = None, heads: int | None = None,
     return {"q": q, "k": k, "v": v, "point": point}
 
 
-def generate_into(w: Workload, q, k, v, seed: int | None = None, threads: int | None = None):
+def generate_into(w: Workload, q, k, v, seed: int | None = None, threads: int | None = None, head0: int = 0):
     """Fill caller-owned host buffers (anything exposing a data pointer of the right size).
 
     q, k, v must be contiguous [heads][S*N][d] arrays of the workload's dtype
@@ -109,7 +111,7 @@ def generate_into(w: Workload, q, k, v, seed: int | None = None, threads: int | 
     cfg = _Cfg(bh, w.frames, w.tokens, w.head_dim, w.n_sink, w.n_points, w.window,
                float(w.p_assign), A_LAT, A_NOISE, SINK_K_SCALE,
                int(w.seed if seed is None else seed), 1 if w.dtype == "bf16" else 0,
-               int(threads or default_threads()))
+               int(threads or default_threads()), int(head0))
     rc = lib.synth_generate(ctypes.byref(cfg), ptr(q), ptr(k), ptr(v), None)
     if rc != 0:
         raise RuntimeError("synth_generate failed with code %d" % rc)

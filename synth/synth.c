@@ -46,6 +46,7 @@ typedef struct {
     uint64_t seed;
     int32_t out_bf16;     /* 1: write bf16 bit patterns (uint16), 0: float32 */
     int32_t n_threads;    /* worker threads (>= 1) */
+    int32_t head0;        /* global index of the first head drawn (a shard of a larger draw) */
 } synth_cfg;
 
 enum { ST_ASSIGN = 1, ST_START = 2, ST_LATENT = 3, ST_QN = 4, ST_KN = 5, ST_VN = 6 };
@@ -157,7 +158,7 @@ static void* head_worker(void* arg) {
         for (int64_t p = j->i0; p < j->i1; ++p)
             for (int64_t e = 0; e < d; e += 2) {
                 double z0, z1;
-                normal_pair(counter(c->seed, ST_LATENT, (uint64_t)j->h, (uint64_t)p, (uint64_t)(e / 2)), &z0,
+                normal_pair(counter(c->seed, ST_LATENT, (uint64_t)(c->head0 + j->h), (uint64_t)p, (uint64_t)(e / 2)), &z0,
                             &z1);
                 j->latent[p * d + e] = (float)z0;
                 j->latent[p * d + e + 1] = (float)z1;
@@ -171,9 +172,9 @@ static void* head_worker(void* arg) {
         for (int64_t e = 0; e < d; e += 2) {
             double qn[2], kn[2], vn[2];
             const uint64_t pe = (uint64_t)(e / 2);
-            normal_pair(counter(c->seed, ST_QN, (uint64_t)j->h, (uint64_t)t, pe), &qn[0], &qn[1]);
-            normal_pair(counter(c->seed, ST_KN, (uint64_t)j->h, (uint64_t)t, pe), &kn[0], &kn[1]);
-            normal_pair(counter(c->seed, ST_VN, (uint64_t)j->h, (uint64_t)t, pe), &vn[0], &vn[1]);
+            normal_pair(counter(c->seed, ST_QN, (uint64_t)(c->head0 + j->h), (uint64_t)t, pe), &qn[0], &qn[1]);
+            normal_pair(counter(c->seed, ST_KN, (uint64_t)(c->head0 + j->h), (uint64_t)t, pe), &kn[0], &kn[1]);
+            normal_pair(counter(c->seed, ST_VN, (uint64_t)(c->head0 + j->h), (uint64_t)t, pe), &vn[0], &vn[1]);
             for (int r = 0; r < 2; ++r) {
                 double qv, kv;
                 if (p >= 0) {
@@ -222,6 +223,7 @@ static int run_parallel(void* (*fn)(void*), void* jobs, size_t job_size, int n) 
 int synth_generate(const synth_cfg* c, void* q, void* k, void* v, int32_t* point_of_token) {
     if (!c || !q || !k || !v) return -1;
     if (c->bh <= 0 || c->frames <= 0 || c->tokens <= 0 || c->head_dim <= 0 || (c->head_dim & 1)) return -2;
+    if (c->head0 < 0 || c->head0 + c->bh > 256) return -2; /* the counter holds 8 bits of head */
     if (c->n_points <= 0 || c->n_sink < 0 || c->window < 0 || c->window > c->frames) return -3;
     if ((int64_t)c->frames * c->tokens >= (1ll << 22) || c->n_points >= (1 << 22) || c->bh > 255) return -4;
     const int nth = c->n_threads > 0 ? c->n_threads : 1;

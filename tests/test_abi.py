@@ -69,6 +69,12 @@ def test_validation_happens_before_any_launch(lib):
     assert lib.sa_select_topk(s, fake, None, None, -1, fake, fake, 20, None, 0, None) == sa.SA_ERR_INVALID_ARG
     # streamed selection without its workspace
     assert lib.sa_select_topk(s, None, fake, fake, 3, fake, fake, 20, None, 0, None) == sa.SA_ERR_WORKSPACE
+    # per-head budgets: no budget array, a misaligned one, a negative bound, a list too short for the bound
+    assert lib.sa_select_topk_per_head(s, fake, None, None, None, 3, fake, fake, 20, None, 0, None) == sa.SA_ERR_INVALID_ARG
+    odd2 = P(0x10002)
+    assert lib.sa_select_topk_per_head(s, fake, None, None, odd2, 3, fake, fake, 20, None, 0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_select_topk_per_head(s, fake, None, None, fake, -1, fake, fake, 20, None, 0, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_select_topk_per_head(s, fake, None, None, fake, 3, fake, fake, 2, None, 0, None) == sa.SA_ERR_INVALID_ARG
     # landmark mode without pools
     assert lib.sa_sparse_attn_fwd(s, fake, fake, fake, fake, fake, 6, fake, fake, 1, None, None, None, None, 0,
                                   fake, None, None) == sa.SA_ERR_INVALID_ARG
@@ -105,3 +111,20 @@ def test_package_fails_loudly_without_library(tmp_path):
         sa._lib = None
         sa.load(str(tmp_path / "missing.so"))
     sa._lib = None
+
+
+def test_sga_host_checks(lib):
+    from view_recon_b200 import sa
+    fake = ctypes.c_void_p(0x10000)
+    shp = sa.shape(2, 4, 5 + 37 * 37, 64, 128, 5, "bf16")
+    s = ctypes.byref(shp)
+    assert lib.sa_sga_workspace_size(s, 37, 37, 3, 3) > 0
+    assert lib.sa_sga_workspace_size(s, 36, 37, 3, 3) == 0        # grid does not match the tokens
+    assert lib.sa_sga_workspace_size(s, 37, 37, 0, 3) == 0        # stride < 1
+    f32 = sa.shape(2, 4, 5 + 37 * 37, 64, 128, 5, "f32")
+    assert lib.sa_sga_workspace_size(ctypes.byref(f32), 37, 37, 3, 3) == 0
+    assert lib.sa_sga_fwd(s, 36, 37, 3, 3, fake, fake, fake, fake, 1 << 40, fake, None, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_sga_fwd(s, 37, 37, 3, 3, None, fake, fake, fake, 1 << 40, fake, None, None) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_sga_fwd(s, 37, 37, 3, 3, fake, fake, fake, fake, 16, fake, None, None) == sa.SA_ERR_WORKSPACE
+    assert lib.sa_sga_fwd(ctypes.byref(f32), 37, 37, 3, 3, fake, fake, fake, fake, 1 << 40, fake, None,
+                          None) == sa.SA_ERR_UNSUPPORTED

@@ -35,6 +35,7 @@ CASES = [
     small("f32_tile128", dtype="f32", frames=2, tokens=300, k=2),
     small("streamed_select", frames=4, tokens=600, k=3, streamed=True),
     small("window_landmark_streamed", frames=6, tokens=500, k=4, landmark=True, streamed=True, window=2),
+    small("one_tile_per_frame", frames=6, tokens=100, k=2, landmark=True),
 ]
 
 
@@ -160,3 +161,73 @@ def test_argument_errors_touch_nothing():
     assert e.value.status == sa.SA_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert torch.equal(before, layer.buf.o)
+
+
+def test_host_pipeline_matches_device_calls():
+    """Overlapped host-input calls give exactly the outputs of plain device calls."""
+    import torch
+    from view_recon_b200.pipeline import HostPipeline, SparseGlobalAttention
+    w = small("hostpipe", frames=3, tokens=700, k=3)
+    make = lambda: SparseGlobalAttention(w.heads, w.frames, w.tokens, w.k, w.tile, w.n_sink, w.dtype)
+    pipe = HostPipeline(make)
+    ref_layer = make()
+    hosts, outs, refs = [], [], []
+    for seed in (1, 2, 3, 4, 5):
+        d = H.inputs(w, seed=seed)
+        hq, hk, hv = (torch.from_numpy(d[x]).view(torch.bfloat16).pin_memory() for x in ("q", "k", "v"))
+        ho = torch.empty_like(hq).pin_memory()
+        hosts.append((hq, hk, hv))
+        outs.append(ho)
+        o, _ = ref_layer.forward(hq.cuda(), hk.cuda(), hv.cuda())
+        refs.append(o.cpu())
+    for (hq, hk, hv), ho in zip(hosts, outs):
+        pipe.submit(hq, hk, hv, ho)
+    pipe.synchronize()
+    for ho, ref in zip(outs, refs):
+        assert torch.equal(ho.view(torch.int16), ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("landmark,streamed", [(False, False), (True, False), (False, True)])
+def test_per_head_budgets(landmark, streamed):
+    """Per-head budgets (one head dense, one frame-only, two in between) through all four steps."""
+    import torch
+    from view_recon_b200 import sa
+    from view_recon_b200.pipeline import SparseGlobalAttention
+    w = small("per_head", frames=5, tokens=700, heads=4, k=3, landmark=landmark, streamed=streamed)
+    g = H.geometry(w)
+    budgets = [0, 2, 99, 7]
+    data = H.inputs(w)
+    q, k, v = (H.to_device(data[x], w.dtype) for x in ("q", "k", "v"))
+    layer = SparseGlobalAttention(w.heads, w.frames, w.tokens, budgets, w.tile, w.n_sink, w.dtype, landmark,
+                                  streamed)
+    layer.forward(q, k, v)
+    torch.cuda.synchronize()
+    assert sa.sa_check_device_error() == 0
+    Q, K, V = (orc.to_f64(data[x]) for x in ("q", "k", "v"))
+    qb, kb, vb, cnt, _, _ = orc.pool(g, Q, K, V)
+    s = orc.scores(qb, kb)
+    kept = H.kept_lists(layer)
+    assert H.from_device(layer.buf.kept_idx).shape[2] == orc.max_kept(g, max(budgets))
+    ref = orc.select_per_head(g, s, budgets)
+    for h, kh in enumerate(budgets):
+        for i in range(g.nt):
+            assert len(kept[h][i]) == len(ref[h][i])
+            ok, msg = orc.selection_matches(g, s[h, i], i, kh, kept[h][i])
+            assert ok, "h=%d i=%d: %s" % (h, i, msg)
+    O_ref, L_ref = orc.attend(g, Q, K, V, kept, 0.125, landmark, kb, vb, cnt)
+    H.check_attention(H.from_device(layer.buf.o), H.from_device(layer.buf.lse), O_ref, L_ref)
+
+
+def test_per_head_budget_out_of_bound_is_reported_and_clamped():
+    import torch
+    from view_recon_b200 import sa
+    w = small("per_head_bad", frames=3, tokens=300, heads=2, k=2, n_sink=0)
+    g = H.geometry(w)
+    layer, _ = H.run_gpu(w, H.inputs(w))
+    torch.cuda.synchronize()
+    bad = torch.tensor([1, 9], dtype=torch.int32, device="cuda")   # 9 > k_max = 2
+    sa.sa_select_topk_per_head(layer.shape, layer.buf.scores, None, None, bad, 2, layer.buf.kept_idx,
+                               layer.buf.kept_cnt, layer.max_kept)
+    assert sa.sa_check_device_error() == sa.SA_ERR_INVALID_ARG
+    cnt = H.from_device(layer.buf.kept_cnt)
+    assert (cnt[0] == g.tpf + 1).all() and (cnt[1] == g.tpf + 2).all()

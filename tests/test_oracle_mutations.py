@@ -18,6 +18,7 @@ PIN_TESTS = [
     lambda: pins.test_scores_closed_form(),
     lambda: pins.test_scores_not_transposed(),
     *[lambda s=s: pins.test_select_bruteforce_subsets(s) for s in range(3)],
+    lambda: pins.test_select_per_head_bruteforce(),
     lambda: pins.test_select_edges(),
     lambda: pins.test_select_skips_keyless_tiles(),
     lambda: pins.test_attention_two_key_closed_form(),
@@ -29,6 +30,8 @@ PIN_TESTS = [
     lambda: pins.test_frame_permutation_equivariance(True),
     lambda: pins.test_landmarks_exact_when_tile_keys_are_identical(),
     lambda: pins.test_k0_is_frame_attention_plus_sinks(),
+    lambda: pins.test_sga_kept_positions(),
+    *[lambda a=a, b=b: pins.test_sga_exact_when_discarded_tokens_are_identical(a, b) for a, b in ((2, 2), (3, 2))],
 ]
 
 
@@ -78,6 +81,61 @@ def select_no_force(g, s_row, i, k):
     cand = np.arange(g.nt)  # slip: own frame competes instead of being forced
     order = np.lexsort((cand, -s_row[cand]))
     return np.sort(cand[order[:orc.max_kept(g, k)]])
+
+
+_select_per_head = orc.select_per_head
+
+
+def per_head_first_budget(g, s, k_per_head):
+    return _select_per_head(g, s, [k_per_head[0]] * s.shape[0])  # slip: one budget for every head
+
+
+def per_head_budgets_shifted(g, s, k_per_head):
+    ks = list(k_per_head)
+    return _select_per_head(g, s, ks[1:] + ks[:1])  # slip: budget of the next head
+
+
+_sga_kept = orc.sga_kept
+
+
+def sga_kept_offset(frames, tokens, n_special, grid_h, grid_w, s_h, s_w):
+    kept = _sga_kept(frames, tokens, n_special, grid_h, grid_w, s_h, s_w)
+    per = kept[:tokens].copy()
+    patches = per[n_special:].reshape(grid_h, grid_w)
+    per[n_special:] = np.roll(patches, (s_h - 1, s_w - 1), axis=(0, 1)).reshape(-1)  # slip: last of each window
+    return np.tile(per, frames)
+
+
+def sga_kept_no_specials(frames, tokens, n_special, grid_h, grid_w, s_h, s_w):
+    kept = _sga_kept(frames, tokens, n_special, grid_h, grid_w, s_h, s_w).reshape(frames, tokens)
+    kept[:, :n_special] = False  # slip: special tokens subsampled away
+    return kept.reshape(-1)
+
+
+def _sga_variant(count_mode="exclude", keep_diagonal=True, bias=True):
+    def sga(q, k, v, frames, tokens, n_special, grid_h, grid_w, s_h, s_w, scale):
+        bh, L, _ = q.shape
+        kept = orc.sga_kept(frames, tokens, n_special, grid_h, grid_w, s_h, s_w)
+        disc = np.nonzero(~kept)[0]
+        kidx = np.nonzero(kept)[0]
+        O = np.zeros((bh, L, v.shape[2]))
+        LSE = np.zeros((bh, L))
+        for h in range(bh):
+            for t in range(L):
+                own = not kept[t]
+                keys, vals = [k[h, kidx]], [v[h, kidx]]
+                if own and keep_diagonal:
+                    keys.append(k[h, t][None]); vals.append(v[h, t][None])
+                others = disc[disc != t] if count_mode == "exclude" else disc
+                lg = [scale * (np.concatenate(keys) @ q[h, t])]
+                if len(others):
+                    kb, vb = k[h, others].mean(axis=0), v[h, others].mean(axis=0)
+                    lg.append(np.array([scale * (kb @ q[h, t]) + (math.log(len(others)) if bias else 0.0)]))
+                    vals.append(vb[None])
+                o, lse = orc._softmax_rows(np.concatenate(lg)[None], np.concatenate(vals))
+                O[h, t], LSE[h, t] = o[0], lse[0]
+        return O, LSE
+    return sga
 
 
 def _attend_variant(bias_sign=1.0, drop_scale=False, drop_sinks=False, bias_inside_scale=False):
@@ -131,11 +189,18 @@ MUTANTS = {
     "ties_to_higher_index": ("select_row", select_ties_high),
     "k_counts_own_frame": ("select_row", select_counts_own_frame),
     "own_frame_not_forced": ("select_row", select_no_force),
+    "per_head_one_budget": ("select_per_head", per_head_first_budget),
+    "per_head_budgets_shifted": ("select_per_head", per_head_budgets_shifted),
     "landmark_bias_negated": ("attend_tile", _attend_variant(bias_sign=-1.0)),
     "scale_dropped": ("attend_tile", _attend_variant(drop_scale=True)),
     "sinks_dropped": ("attend_tile", _attend_variant(drop_sinks=True)),
     "bias_inside_scale": ("attend_tile", _attend_variant(bias_inside_scale=True)),
     "lse_without_max": ("_softmax_rows", softmax_lse_without_max),
+    "sga_grid_offset": ("sga_kept", sga_kept_offset),
+    "sga_specials_dropped": ("sga_kept", sga_kept_no_specials),
+    "sga_count_includes_own_column": ("sga", _sga_variant(count_mode="all")),
+    "sga_diagonal_dropped": ("sga", _sga_variant(keep_diagonal=False)),
+    "sga_no_count_bias": ("sga", _sga_variant(bias=False)),
     "softmax_not_normalised": ("_softmax_rows", softmax_no_normalise),
 }
 

@@ -142,6 +142,35 @@ def test_select_bruteforce_subsets(seed):
             assert orc.select_row(g, s, i, k).tolist() == want
 
 
+def test_select_per_head_bruteforce():
+    """Per-head budgets: each head's lists are the brute-force top-k of that head's row."""
+    g = orc.Geometry(frames=3, tokens=6, tile=2, n_sink=0)  # tpf 3, nt 9, 6 candidates
+    rng = np.random.default_rng(11)
+    budgets = [0, 2, 5, 99]
+    s = rng.integers(-2, 3, size=(len(budgets), g.nt, g.nt)).astype(float)
+    kept = orc.select_per_head(g, s, budgets)
+    for h, k in enumerate(budgets):
+        for i in range(g.nt):
+            cand = [j for j in range(g.nt) if j // 3 != i // 3]
+            kk = min(k, len(cand))
+            winners = [c for c in itertools.combinations(cand, kk) if _is_topk(s[h, i], cand, c)]
+            own = [j for j in range(g.nt) if j // 3 == i // 3]
+            assert kept[h][i].tolist() == sorted(list(winners[0]) + own)
+
+
+def test_selection_is_nested_in_the_budget():
+    """With the (score desc, index asc) order, a larger budget only adds tiles."""
+    g = orc.Geometry(frames=4, tokens=10, tile=4, n_sink=1)  # tpf 3, nt 12
+    rng = np.random.default_rng(5)
+    s = rng.integers(-3, 4, size=(g.nt, g.nt)).astype(float)
+    for i in range(g.nt):
+        prev = set(orc.select_row(g, s[i], i, 0).tolist())
+        for k in range(1, g.nt + 2):
+            cur = set(orc.select_row(g, s[i], i, k).tolist())
+            assert prev <= cur and len(cur) - len(prev) <= 1
+            prev = cur
+
+
 def test_select_edges():
     g = orc.Geometry(frames=4, tokens=4, tile=2, n_sink=0)  # tpf 2, nt 8
     s = np.zeros(g.nt)
@@ -331,3 +360,40 @@ def test_k0_is_frame_attention_plus_sinks():
         keys = [f * 6 + n for n in range(2, 6)] + sinks
         o, _ = _textbook_row(q[0, t], k[0, keys].tolist(), v[0, keys].tolist(), 0.3)
         np.testing.assert_allclose(O[0, t], o, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- subsampled global attention
+
+def test_sga_kept_positions():
+    # one frame: 2 special tokens, then a 3 x 5 grid; stride (2, 2) keeps rows 0, 2 and columns 0, 2, 4
+    kept = orc.sga_kept(frames=2, tokens=2 + 15, n_special=2, grid_h=3, grid_w=5, s_h=2, s_w=2)
+    per = [0, 1] + [2 + r * 5 + c for r in (0, 2) for c in (0, 2, 4)]
+    assert np.nonzero(kept)[0].tolist() == per + [17 + j for j in per]
+
+
+@pytest.mark.parametrize("n_special,gh,gw", [(0, 3, 4), (2, 4, 5)])
+def test_sga_stride_one_is_dense(n_special, gh, gw):
+    rng = np.random.default_rng(3)
+    S, N = 2, n_special + gh * gw
+    q, k, v = (rng.standard_normal((2, S * N, 8)) for _ in range(3))
+    O, LSE = orc.sga(q, k, v, S, N, n_special, gh, gw, 1, 1, 0.3)
+    Od, Ld = orc.dense(q, k, v, 0.3)
+    assert np.abs(O - Od).max() < 1e-12 and np.abs(LSE - Ld).max() < 1e-12
+
+
+@pytest.mark.parametrize("s_h,s_w", [(2, 2), (3, 2), (4, 5)])
+def test_sga_exact_when_discarded_tokens_are_identical(s_h, s_w):
+    """The mean pair stands for the discarded columns exactly when they are all equal: then the
+    layer equals dense attention (this pins the ln(count) bias, the diagonal, and the count
+    excluding the query's own discarded column)."""
+    rng = np.random.default_rng(4)
+    S, ns, gh, gw = 3, 2, 5, 7
+    N = ns + gh * gw
+    q, k, v = (rng.standard_normal((2, S * N, 8)) for _ in range(3))
+    kept = orc.sga_kept(S, N, ns, gh, gw, s_h, s_w)
+    for h in range(2):
+        k[h, ~kept] = rng.standard_normal(8)
+        v[h, ~kept] = rng.standard_normal(8)
+    O, LSE = orc.sga(q, k, v, S, N, ns, gh, gw, s_h, s_w, 0.25)
+    Od, Ld = orc.dense(q, k, v, 0.25)
+    assert np.abs(O - Od).max() < 1e-12 and np.abs(LSE - Ld).max() < 1e-12

@@ -68,3 +68,15 @@ def test_visibility_window():
             frames_of.setdefault(int(pt), set()).add(t // w.tokens)
     assert frames_of
     assert max(max(f) - min(f) for f in frames_of.values()) <= w.window - 1
+
+
+def test_head_shard_is_a_slice_of_the_full_draw():
+    import numpy as np
+    import synth
+    from synth.workloads import TINY, VGGT_S16
+    for w in (TINY, VGGT_S16.scaled(frames=2)):
+        full = synth.generate(w, heads=4)
+        part = synth.generate(w, heads=2, head0=1)
+        for x in ("q", "k", "v"):
+            assert np.array_equal(part[x], full[x][1:3])
+        assert np.array_equal(part["point"], full["point"])

@@ -42,11 +42,12 @@ struct __align__(64) TcArgs {
     float* lse;
     int32_t max_kept;
     int32_t frames, tokens, n_sink, tpf, nt, L, ntp;
+    int32_t Lk;        // dense: key rows per head (L, or the length of a compacted key sequence)
     int32_t n_vtiles;  // transposed V tiles per head (nt, or ceil(L/128) dense)
     int32_t n_sink_rows, n_sink_tiles, n_lm_chunks;
     int32_t dense, landmark;
     int32_t q_per_head, total_items;
-    uint32_t tpf_magic;  // j / tpf == __umulhi(j, tpf_magic) for every tile index j < nt
+    uint32_t tpf_magic;  // j / tpf == __umulhi(j, tpf_magic) for every tile index j < nt (tpf > 1)
     float scale_log2;
 };
 
@@ -90,7 +91,7 @@ __device__ __forceinline__ Slot make_slot(const TcArgs& a, int item) {
     if (a.dense) {
         s.qrow = s.h * a.L + s.i * 128;
         s.nq = min(128, a.L - s.i * 128);
-        s.n_items = s.active ? (a.L + 127) / 128 : 0;
+        s.n_items = s.active ? (a.Lk + 127) / 128 : 0;
     } else {
         const int f = s.i / a.tpf, slot = s.i % a.tpf;
         s.qrow = s.h * a.L + f * a.tokens + slot * 128;
@@ -118,10 +119,10 @@ __device__ __forceinline__ Item get_item_j(const TcArgs& a, const Slot& s, int n
     it.chunk = 0;
     if (a.dense) {
         it.kind = 0;
-        it.krow = s.h * a.L + n * 128;
+        it.krow = s.h * a.Lk + n * 128;
         it.vrow = (s.h * a.n_vtiles + n) * 64;
         it.lo = 0;
-        it.hi = min(128, a.L - n * 128);
+        it.hi = min(128, a.Lk - n * 128);
         return it;
     }
     if (n < s.cnt) {
@@ -132,7 +133,7 @@ __device__ __forceinline__ Item get_item_j(const TcArgs& a, const Slot& s, int n
             it.lo = it.hi = 0;
             return it;
         }
-        const int f = (int)__umulhi((uint32_t)j, a.tpf_magic), slot = j - f * a.tpf;
+        const int f = a.tpf == 1 ? j : (int)__umulhi((uint32_t)j, a.tpf_magic), slot = j - f * a.tpf;
         const int n0 = slot * 128;
         const int nk = min(128, a.tokens - n0);
         it.kind = 0;
@@ -384,10 +385,7 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv + 32);
             uint32_t(&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv + 64);
             uint32_t(&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv + 96);
-            tmem_ld_32x32b_x32(tS + 0, s0);
-            tmem_ld_32x32b_x32(tS + 32, s1);
-            tmem_ld_32x32b_x32(tS + 64, s2);
-            tmem_ld_32x32b_x32(tS + 96, s3);
+            tmem_ld_32x32b_x128(tS, sv);
             tmem_ld_wait(s0);
             reg_fence(s1);
             reg_fence(s2);

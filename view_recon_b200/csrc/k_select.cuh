@@ -38,7 +38,17 @@ struct SelectArgs {
     int32_t nt, tpf, tile, tokens, n_sink;
     int32_t k, max_kept;
     int32_t h0, i0, rows;
+    const int32_t* k_head;  // per-head budgets [bh] (device), or null: every head uses k
+    int32_t k_max;          // bound on every k_head entry (max_kept was checked against it)
 };
+
+// Budget of head h: k, or k_head[h] clamped to [0, k_max] (an entry outside is reported).
+__device__ __forceinline__ uint32_t sel_budget(const SelectArgs& a, int h, bool reporter) {
+    if (!a.k_head) return (uint32_t)max(a.k, 0);
+    const int kh = __ldg(a.k_head + h);
+    if ((kh < 0 || kh > a.k_max) && reporter) sa_flag_error(SA_ERR_INVALID_ARG);
+    return (uint32_t)min(max(kh, 0), a.k_max);
+}
 
 // Shared memory of one warp, in words: the row (4 words of slack so that its 16-byte-aligned
 // middle lands 16-byte aligned), the histogram, the gathered keys.
@@ -183,7 +193,7 @@ __global__ void __launch_bounds__(32 * SEL_MAX_WARPS) select_topk_warp_kernel(Se
         __syncwarp();
     }
 
-    const uint32_t k_req = (uint32_t)max(a.k, 0);
+    const uint32_t k_req = sel_budget(a, h, lane == 0);
     const SelBin b1 = sel_find_bin_warp<SEL_H1>(hist, k_req);
     const uint32_t ncand = b1.total;
     const uint32_t kk = min(k_req, ncand);
@@ -427,7 +437,7 @@ __global__ void __launch_bounds__(SEL_BLOCK_THREADS) select_topk_block_kernel(Se
         }
         __syncthreads();
     }
-    const uint32_t k_req = (uint32_t)max(a.k, 0);
+    const uint32_t k_req = sel_budget(a, h, tid == 0);
     const uint32_t ncand = sel_find_bin<SEL_BLOCK_H1 / SEL_BLOCK_THREADS>(hist1, k_req, scratch, &sb);
     const uint32_t kk = min(k_req, ncand);
     // selected: own frame, or (key >> shift) > prefix, or == prefix and admitted; with

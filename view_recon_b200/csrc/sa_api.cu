@@ -11,6 +11,7 @@
 #include "k_pool.cuh"
 #include "k_scores.cuh"
 #include "k_select.cuh"
+#include "k_sga.cuh"
 
 // Fixed scratch of sa_select_topk_noalloc: one block of score rows (2 Mi floats = 8 MiB).
 constexpr long long kNoallocScratchFloats = 1ll << 21;
@@ -196,11 +197,13 @@ struct AttnWs {
     int64_t n_vtiles, n_sink_tiles, n_lm_chunks, ntp;
     size_t vt, svt, lk, lvt, lbias, total;
 };
-AttnWs attn_ws(const Geo& g, bool dense, bool landmark) {
+// Lk: key rows per head in dense mode (g.L, or the length of a compacted key sequence).
+AttnWs attn_ws(const Geo& g, bool dense, bool landmark, int64_t Lk = -1) {
     AttnWs w;
     constexpr size_t kTile = 64 * 128 * 2;
+    if (Lk < 0) Lk = g.L;
     w.ntp = (g.nt + 127) / 128 * 128;
-    w.n_vtiles = dense ? (g.L + 127) / 128 : g.nt;
+    w.n_vtiles = dense ? (Lk + 127) / 128 : g.nt;
     w.n_sink_tiles = dense ? 0 : (g.S * g.n_sink + 127) / 128;
     w.n_lm_chunks = (!dense && landmark) ? w.ntp / 128 : 0;
     size_t off = 0;
@@ -230,17 +233,19 @@ size_t select_rows_per_block(const Geo& g) {
 sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v, const int32_t* kept_idx,
                       const int32_t* kept_cnt, int32_t max_kept, const void* sink_k, const void* sink_v,
                       int32_t landmark, const float* k_pool, const float* v_pool, const int32_t* k_cnt,
-                      void* ws, size_t ws_bytes, void* o, float* lse, bool dense, cudaStream_t stream) {
+                      void* ws, size_t ws_bytes, void* o, float* lse, bool dense, cudaStream_t stream,
+                      int64_t Lk = -1) {
     sa_status st = ensure_attributes();
     if (st != SA_OK) return st;
+    if (Lk < 0) Lk = g.L;
     if (use_tc(g)) {
         TcArgs a;
         memset(&a, 0, sizeof(a));
-        const AttnWs w = attn_ws(g, dense, landmark != 0);
+        const AttnWs w = attn_ws(g, dense, landmark != 0, Lk);
         if (!ws || ws_bytes < w.total) return SA_ERR_WORKSPACE;
         uint8_t* base = static_cast<uint8_t*>(ws);
         const int64_t n_sink_rows = g.S * g.n_sink;
-        bool ok = encode_rows_bf16(&a.tm_q, q, g.bh * g.L) && encode_rows_bf16(&a.tm_k, k, g.bh * g.L) &&
+        bool ok = encode_rows_bf16(&a.tm_q, q, g.bh * g.L) && encode_rows_bf16(&a.tm_k, k, g.bh * Lk) &&
                   encode_vt_tiles(&a.tm_vt, base + w.vt, g.bh * w.n_vtiles);
         if (w.n_sink_tiles > 0)
             ok = ok && encode_rows_bf16(&a.tm_sk, sink_k, g.bh * n_sink_rows) &&
@@ -265,7 +270,7 @@ sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v,
             t.tokens = (int32_t)g.N;
             t.tpf = (int32_t)g.tpf;
             t.L = (int32_t)g.L;
-            t.rows_per_head = (int32_t)g.L;
+            t.rows_per_head = (int32_t)Lk;
             if (w.n_vtiles > 2147483647 || g.bh > 65535) return SA_ERR_UNSUPPORTED;
             vtile_transpose_kernel<<<dim3((unsigned)w.n_vtiles, (unsigned)g.bh), 256, 0, stream>>>(t);
             if ((st = launch_status()) != SA_OK) return st;
@@ -299,6 +304,7 @@ sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v,
         a.tpf = (int32_t)g.tpf;
         a.nt = (int32_t)g.nt;
         a.L = (int32_t)g.L;
+        a.Lk = (int32_t)Lk;
         a.ntp = (int32_t)w.ntp;
         a.n_vtiles = (int32_t)w.n_vtiles;
         a.n_sink_rows = (int32_t)n_sink_rows;
@@ -315,10 +321,14 @@ sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v,
             if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
             if (!g_tc_regs_ok[dev]) return SA_ERR_UNSUPPORTED;
         }
-        // exact division by tpf with a multiply-high, checked for every tile index
-        a.tpf_magic = (uint32_t)((0x100000000ull + (uint64_t)g.tpf - 1) / (uint64_t)g.tpf);
-        for (int64_t j = 0; j < g.nt; ++j)
-            if ((int64_t)(((uint64_t)j * a.tpf_magic) >> 32) != j / g.tpf) return SA_ERR_UNSUPPORTED;
+        // exact division by tpf with a multiply-high (tpf > 1; one tile per frame needs none),
+        // checked for every tile index; the dense modes never divide
+        a.tpf_magic = 0;
+        if (!dense && g.tpf > 1) {
+            a.tpf_magic = (uint32_t)((0x100000000ull + (uint64_t)g.tpf - 1) / (uint64_t)g.tpf);
+            for (int64_t j = 0; j < g.nt; ++j)
+                if ((int64_t)(((uint64_t)j * a.tpf_magic) >> 32) != j / g.tpf) return SA_ERR_UNSUPPORTED;
+        }
         const size_t smem = Lay::smem_bytes();
         if (smem > 227 * 1024) return SA_ERR_UNSUPPORTED;
         const int grid = (a.total_items + kTcSlots - 1) / kTcSlots;
@@ -517,9 +527,12 @@ static void launch_select(const SelectArgs& a, unsigned gy, cudaStream_t stream)
     }
 }
 
-sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, const float* q_pool,
-                         const float* k_pool, int32_t k, int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
-                         void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream) {
+// Shared by sa_select_topk (k_head == nullptr: every head keeps k) and
+// sa_select_topk_per_head (head h keeps k_head[h] <= k).
+static sa_status select_impl(const sa_shape* shape, const float* scores_or_null, const float* q_pool,
+                             const float* k_pool, int32_t k, const int32_t* k_head, int32_t* kept_idx,
+                             int32_t* kept_cnt, int32_t max_kept, void* workspace_or_null, size_t workspace_bytes,
+                             sa_stream_t stream) {
     Geo g;
     sa_status st = geo_of(shape, &g);
     if (st != SA_OK) return st;
@@ -545,6 +558,8 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, con
     a.n_sink = (int32_t)g.n_sink;
     a.k = k;
     a.max_kept = max_kept;
+    a.k_head = k_head;
+    a.k_max = k;
     if (scores_or_null) {
         a.scores = scores_or_null;
         a.lds = g.nt;
@@ -584,6 +599,22 @@ sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, con
     return SA_OK;
 }
 
+sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, const float* q_pool,
+                         const float* k_pool, int32_t k, int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
+                         void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream) {
+    return select_impl(shape, scores_or_null, q_pool, k_pool, k, nullptr, kept_idx, kept_cnt, max_kept,
+                       workspace_or_null, workspace_bytes, stream);
+}
+
+sa_status sa_select_topk_per_head(const sa_shape* shape, const float* scores_or_null, const float* q_pool,
+                                  const float* k_pool, const int32_t* k_per_head, int32_t k_max, int32_t* kept_idx,
+                                  int32_t* kept_cnt, int32_t max_kept, void* workspace_or_null,
+                                  size_t workspace_bytes, sa_stream_t stream) {
+    if (!k_per_head || (reinterpret_cast<uintptr_t>(k_per_head) & 3u) || k_max < 0) return SA_ERR_INVALID_ARG;
+    return select_impl(shape, scores_or_null, q_pool, k_pool, k_max, k_per_head, kept_idx, kept_cnt, max_kept,
+                       workspace_or_null, workspace_bytes, stream);
+}
+
 sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, const float* k_pool, int32_t k,
                                  int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept, sa_stream_t stream) {
     Geo g;
@@ -608,6 +639,8 @@ sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, con
     a.n_sink = (int32_t)g.n_sink;
     a.k = k;
     a.max_kept = max_kept;
+    a.k_head = nullptr;
+    a.k_max = k;
     for (int64_t h = 0; h < g.bh; ++h) {
         for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
             const int64_t rows = std::min<int64_t>(R, g.nt - i0);
@@ -693,6 +726,111 @@ sa_status sa_dense_attn_fwd(const sa_shape* shape, const void* q, const void* k,
         return SA_ERR_WORKSPACE;
     return attn_common(g, q, k, v, nullptr, nullptr, 0, nullptr, nullptr, 0, nullptr, nullptr, nullptr,
                        workspace_or_null, workspace_bytes, o, lse_or_null, true, stream);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ subsampled global attention
+
+struct SgaWs {
+    SgaGeo sg;
+    int64_t Lk, n_disc;
+    size_t ksub, vsub, part, sums, lse, attn, attn_bytes, total;
+};
+
+static sa_status sga_plan(const Geo& g, int32_t grid_h, int32_t grid_w, int32_t s_h, int32_t s_w, SgaWs* w) {
+    if (grid_h < 1 || grid_w < 1 || s_h < 1 || s_w < 1) return SA_ERR_INVALID_ARG;
+    if ((int64_t)g.n_sink + (int64_t)grid_h * grid_w != g.N) return SA_ERR_INVALID_ARG;
+    SgaGeo& sg = w->sg;
+    sg.frames = (int32_t)g.S;
+    sg.tokens = (int32_t)g.N;
+    sg.n_special = (int32_t)g.n_sink;
+    sg.grid_h = grid_h;
+    sg.grid_w = grid_w;
+    sg.s_h = s_h;
+    sg.s_w = s_w;
+    sg.kh = (grid_h + s_h - 1) / s_h;
+    sg.kw = (grid_w + s_w - 1) / s_w;
+    sg.kpf = sg.n_special + sg.kh * sg.kw;
+    w->Lk = g.S * sg.kpf;
+    w->n_disc = g.S * ((int64_t)grid_h * grid_w - (int64_t)sg.kh * sg.kw);
+    size_t off = 0;
+    w->ksub = off;
+    off += align256((size_t)g.bh * w->Lk * 128);
+    w->vsub = off;
+    off += align256((size_t)g.bh * w->Lk * 128);
+    w->part = off;
+    off += align256((size_t)g.bh * g.S * 128 * 4);
+    w->sums = off;
+    off += align256((size_t)g.bh * 128 * 4);
+    w->lse = off;
+    off += align256((size_t)g.bh * g.L * 4);
+    w->attn = off;
+    w->attn_bytes = attn_ws(g, true, false, w->Lk).total;
+    off += align256(w->attn_bytes);
+    w->total = off;
+    return SA_OK;
+}
+
+extern "C" {
+
+size_t sa_sga_workspace_size(const sa_shape* shape, int32_t grid_h, int32_t grid_w, int32_t s_h, int32_t s_w) {
+    Geo g;
+    SgaWs w;
+    if (geo_of(shape, &g) != SA_OK || !use_tc(g)) return 0;
+    if (sga_plan(g, grid_h, grid_w, s_h, s_w, &w) != SA_OK) return 0;
+    return w.total;
+}
+
+sa_status sa_sga_fwd(const sa_shape* shape, int32_t grid_h, int32_t grid_w, int32_t s_h, int32_t s_w, const void* q,
+                     const void* k, const void* v, void* workspace, size_t workspace_bytes, void* o, float* lse_or_null,
+                     sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    if (!q || !k || !v || !o) return SA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse_or_null && !aligned16(lse_or_null)))
+        return SA_ERR_INVALID_ARG;
+    SgaWs w;
+    if ((st = sga_plan(g, grid_h, grid_w, s_h, s_w, &w)) != SA_OK) return st;
+    if (!use_tc(g)) return SA_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return SA_ERR_WORKSPACE;
+    if (g.bh > 65535 || g.S > 2147483647 || w.Lk > 2147483647 || g.bh * g.L > (1ll << 40)) return SA_ERR_UNSUPPORTED;
+    if ((st = ensure_attributes()) != SA_OK) return st;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    SgaGatherArgs ga;
+    ga.k = static_cast<const uint32_t*>(k);
+    ga.v = static_cast<const uint32_t*>(v);
+    ga.ksub = reinterpret_cast<uint32_t*>(base + w.ksub);
+    ga.vsub = reinterpret_cast<uint32_t*>(base + w.vsub);
+    ga.part = reinterpret_cast<float*>(base + w.part);
+    ga.L = (int32_t)g.L;
+    ga.Lk = (int32_t)w.Lk;
+    ga.g = w.sg;
+    sga_gather_kernel<<<dim3((unsigned)g.S, (unsigned)g.bh), 256, 0, stream>>>(ga);
+    if ((st = launch_status()) != SA_OK) return st;
+    float* sums = reinterpret_cast<float*>(base + w.sums);
+    sga_sum_kernel<<<(unsigned)g.bh, 128, 0, stream>>>(ga.part, sums, (int32_t)g.S);
+    if ((st = launch_status()) != SA_OK) return st;
+    float* lse_att = reinterpret_cast<float*>(base + w.lse);
+    st = attn_common(g, q, ga.ksub, ga.vsub, nullptr, nullptr, 0, nullptr, nullptr, 0, nullptr, nullptr, nullptr,
+                     base + w.attn, w.attn_bytes, o, lse_att, true, stream, w.Lk);
+    if (st != SA_OK) return st;
+    SgaCombineArgs ca;
+    ca.q = static_cast<const uint32_t*>(q);
+    ca.k = static_cast<const uint32_t*>(k);
+    ca.v = static_cast<const uint32_t*>(v);
+    ca.o = static_cast<uint32_t*>(o);
+    ca.lse_in = lse_att;
+    ca.lse_out = lse_or_null;
+    ca.sums = sums;
+    ca.rows = g.bh * g.L;
+    ca.L = (int32_t)g.L;
+    ca.n_disc = (int32_t)w.n_disc;
+    ca.scale = g.scale;
+    ca.g = w.sg;
+    sga_combine_kernel<<<(unsigned)((ca.rows + 7) / 8), 256, 0, stream>>>(ca);
+    return launch_status();
 }
 
 }  // extern "C"

@@ -37,7 +37,9 @@ class Buffers:
 class SparseGlobalAttention:
     """Dynamic tile-sparse global attention for bh heads of S frames x N tokens (d = 64).
 
-    k          key tiles chosen per query tile beyond its own frame's tiles
+    k          key tiles chosen per query tile beyond its own frame's tiles: one budget for every
+               head, or a sequence of bh per-head budgets (a budget at or above the candidate
+               count makes that head dense)
     landmark   fold every unselected tile into one mean-K/mean-V token (+ln count bias)
     streamed   select without materialising the [bh][nt][nt] score matrix
     """
@@ -47,7 +49,13 @@ class SparseGlobalAttention:
                  device=None, with_lse: bool = True):
         import torch
         self.shape = sa.shape(bh, frames, tokens, head_dim, tile, n_sink, dtype)
-        self.k = int(k)
+        if isinstance(k, (int,)) or getattr(k, "ndim", None) == 0:
+            self.k, self.k_per_head = int(k), None
+        else:
+            ks = [int(x) for x in k]
+            if len(ks) != bh or min(ks) < 0:
+                raise ValueError("k needs one non-negative budget per head")
+            self.k, self.k_per_head = max(ks), ks
         self.landmark = bool(landmark)
         self.streamed = bool(streamed)
         self.nt = sa.sa_num_tiles(self.shape)
@@ -64,6 +72,8 @@ class SparseGlobalAttention:
         nt = self.nt
         sel_bytes = sa.sa_select_workspace_size(self.shape, self.streamed)
         attn_bytes = sa.sa_sparse_attn_workspace_size(self.shape, self.landmark)
+        self.k_head = (torch.tensor(self.k_per_head, dtype=torch.int32, device=dev)
+                       if self.k_per_head is not None else None)
         self.buf = Buffers(
             q_pool=torch.empty((bh, nt, head_dim), dtype=f32, device=dev),
             k_pool=torch.empty((bh, nt, head_dim), dtype=f32, device=dev),
@@ -91,8 +101,12 @@ class SparseGlobalAttention:
 
     def select(self, stream=None):
         b = self.buf
-        sa.sa_select_topk(self.shape, b.scores, b.q_pool, b.k_pool, self.k, b.kept_idx, b.kept_cnt,
-                          self.max_kept, b.sel_ws, stream)
+        if self.k_head is None:
+            sa.sa_select_topk(self.shape, b.scores, b.q_pool, b.k_pool, self.k, b.kept_idx, b.kept_cnt,
+                              self.max_kept, b.sel_ws, stream)
+        else:
+            sa.sa_select_topk_per_head(self.shape, b.scores, b.q_pool, b.k_pool, self.k_head, self.k, b.kept_idx,
+                                       b.kept_cnt, self.max_kept, b.sel_ws, stream)
 
     def attend(self, q, k, v, stream=None):
         b = self.buf
@@ -125,6 +139,91 @@ class SparseGlobalAttention:
             if self.landmark:
                 n += 1  # landmark tables
         return n
+
+
+class HostPipeline:
+    """Layer calls on host-resident (pinned) Q/K/V with the transfers overlapped.
+
+    Two layer objects and two sets of device inputs alternate between calls; three streams
+    carry the host-to-device copies, the four C-ABI steps and the device-to-host copy of O, so
+    that the copy-in of call i+1 and the copy-out of call i-1 run while call i computes.
+    `make_layer` builds one `SparseGlobalAttention`; inputs are [bh][L][d] host tensors.
+    """
+
+    def __init__(self, make_layer):
+        import torch
+        self.layers = [make_layer(), make_layer()]
+        lay = self.layers[0]
+        shape = (lay.bh, lay.L, lay.d)
+        self.dev_in = [[torch.empty(shape, dtype=lay.dtype, device=lay.device) for _ in range(3)] for _ in range(2)]
+        self.s_in = torch.cuda.Stream(lay.device)
+        self.s_comp = torch.cuda.Stream(lay.device)
+        self.s_out = torch.cuda.Stream(lay.device)
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer set s are on the device
+        self.ev_comp = [torch.cuda.Event() for _ in range(2)]  # the layer of set s has finished
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]   # O of set s has left the device
+        self.calls = 0
+
+    def submit(self, hq, hk, hv, ho):
+        """Queue one call: hq, hk, hv pinned host inputs, ho the pinned host output."""
+        import torch
+        s = self.calls % 2
+        self.calls += 1
+        dq, dk, dv = self.dev_in[s]
+        self.s_in.wait_event(self.ev_comp[s])  # the call two back has consumed these buffers
+        with torch.cuda.stream(self.s_in):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+        self.ev_in[s].record(self.s_in)
+        self.s_comp.wait_event(self.ev_in[s])
+        self.s_comp.wait_event(self.ev_out[s])  # O of the call two back has been copied out
+        o, _ = self.layers[s].forward(dq, dk, dv, stream=self.s_comp)
+        self.ev_comp[s].record(self.s_comp)
+        self.s_out.wait_event(self.ev_comp[s])
+        with torch.cuda.stream(self.s_out):
+            ho.copy_(o, non_blocking=True)
+        self.ev_out[s].record(self.s_out)
+
+    def synchronize(self):
+        self.s_out.synchronize()
+        self.s_comp.synchronize()
+        self.s_in.synchronize()
+
+
+class SubsampledGlobalAttention:
+    """Subsampled global attention (AVGGT SGA) for bh heads of S frames x N tokens, N = n_special +
+    grid_h * grid_w: keys/values kept on a stride_h x stride_w grid of each frame's patches plus
+    every special token, each token's own key, and one mean pair for the other discarded tokens.
+    One C call (sa_sga_fwd); the workspace is allocated once."""
+
+    def __init__(self, bh: int, frames: int, tokens: int, grid=(37, 37), stride=(3, 3), n_special: int = 5,
+                 dtype: str = "bf16", head_dim: int = 64, device=None, with_lse: bool = True):
+        import torch
+        self.shape = sa.shape(bh, frames, tokens, head_dim, 128, n_special, dtype)
+        self.grid = (int(grid[0]), int(grid[1]))
+        self.stride = (int(stride[0]), int(stride[1]))
+        nbytes = sa.sa_sga_workspace_size(self.shape, *self.grid, *self.stride)
+        if nbytes == 0:
+            raise ValueError("unsupported shape or grid for subsampled global attention")
+        dev = torch.device(device if device is not None else "cuda")
+        self.bh, self.frames, self.tokens, self.d = bh, frames, tokens, head_dim
+        self.L = frames * tokens
+        self.device = dev
+        self.ws = torch.empty((nbytes,), dtype=torch.uint8, device=dev)
+        tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.dtype = tdt
+        kh = -(-self.grid[0] // self.stride[0])
+        kw = -(-self.grid[1] // self.stride[1])
+        self.kept_keys = frames * (n_special + kh * kw)  # compacted key sequence per head
+        self.o = torch.empty((bh, self.L, head_dim), dtype=tdt, device=dev)
+        self.lse = torch.empty((bh, self.L), dtype=torch.float32, device=dev) if with_lse else None
+
+    def forward(self, q, k, v, stream=None):
+        sa.sa_sga_fwd(self.shape, *self.grid, *self.stride, q, k, v, self.ws, self.o, self.lse, stream)
+        return self.o, self.lse
+
+    __call__ = forward
 
 
 def dense_attention(q, k, v, frames: int, tokens: int, dtype: str = "bf16", with_lse: bool = True, stream=None):

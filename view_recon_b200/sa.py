@@ -28,8 +28,8 @@ SA_BF16 = 1
 # every symbol include/sa.h declares
 EXPORTS = [
     "sa_num_tiles", "sa_max_kept", "sa_tile_pool", "sa_tile_scores", "sa_select_workspace_size",
-    "sa_select_topk", "sa_select_topk_noalloc", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
-    "sa_dense_attn_fwd",
+    "sa_select_topk", "sa_select_topk_per_head", "sa_select_topk_noalloc", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
+    "sa_dense_attn_fwd", "sa_sga_workspace_size", "sa_sga_fwd",
     "sa_status_string", "sa_check_device_error", "sa_set_wait_limit_ns", "sa_test_withhold_query_load",
 ]
 
@@ -74,6 +74,7 @@ def load(path: str | None = None):
         "sa_tile_scores": (i32, [shp, vp, vp, vp, vp]),
         "sa_select_workspace_size": (sz, [shp, i32]),
         "sa_select_topk": (i32, [shp, vp, vp, vp, i32, vp, vp, i32, vp, sz, vp]),
+        "sa_select_topk_per_head": (i32, [shp, vp, vp, vp, vp, i32, vp, vp, i32, vp, sz, vp]),
         "sa_select_topk_noalloc": (i32, [shp, vp, vp, i32, vp, vp, i32, vp]),
         "sa_sparse_attn_workspace_size": (sz, [shp, i32]),
         "sa_sparse_attn_fwd": (i32, [shp, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp, vp,
@@ -83,6 +84,8 @@ def load(path: str | None = None):
         "sa_status_string": (ctypes.c_char_p, [i32]),
         "sa_check_device_error": (i32, [vp]),
         "sa_set_wait_limit_ns": (i32, [ctypes.c_int64]),
+        "sa_sga_workspace_size": (sz, [shp, i32, i32, i32, i32]),
+        "sa_sga_fwd": (i32, [shp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp, vp]),
         "sa_test_withhold_query_load": (i32, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -161,6 +164,16 @@ def sa_select_topk(shp, scores, q_pool, k_pool, k, kept_idx, kept_cnt, max_kept,
     _check("sa_select_topk", st)
 
 
+def sa_select_topk_per_head(shp, scores, q_pool, k_pool, k_per_head, k_max, kept_idx, kept_cnt, max_kept,
+                            workspace=None, stream=None):
+    """k_per_head: int32 device tensor [bh]."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().sa_select_topk_per_head(ctypes.byref(shp), _ptr(scores), _ptr(q_pool), _ptr(k_pool),
+                                        _ptr(k_per_head), int(k_max), _ptr(kept_idx), _ptr(kept_cnt),
+                                        int(max_kept), _ptr(workspace), ws_bytes, _stream(stream))
+    _check("sa_select_topk_per_head", st)
+
+
 def sa_select_topk_noalloc(shp, q_pool, k_pool, k, kept_idx, kept_cnt, max_kept, stream=None):
     st = load().sa_select_topk_noalloc(ctypes.byref(shp), _ptr(q_pool), _ptr(k_pool), int(k), _ptr(kept_idx),
                                        _ptr(kept_cnt), int(max_kept), _stream(stream))
@@ -202,3 +215,14 @@ def sa_set_wait_limit_ns(limit_ns: int):
 
 def sa_test_withhold_query_load(enable: bool):
     _check("sa_test_withhold_query_load", load().sa_test_withhold_query_load(1 if enable else 0))
+
+
+def sa_sga_workspace_size(shp, grid_h, grid_w, s_h, s_w) -> int:
+    return int(load().sa_sga_workspace_size(ctypes.byref(shp), int(grid_h), int(grid_w), int(s_h), int(s_w)))
+
+
+def sa_sga_fwd(shp, grid_h, grid_w, s_h, s_w, q, k, v, workspace, o, lse=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().sa_sga_fwd(ctypes.byref(shp), int(grid_h), int(grid_w), int(s_h), int(s_w), _ptr(q), _ptr(k),
+                           _ptr(v), _ptr(workspace), ws_bytes, _ptr(o), _ptr(lse), _stream(stream))
+    _check("sa_sga_fwd", st)
