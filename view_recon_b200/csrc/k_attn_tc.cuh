@@ -193,8 +193,8 @@ struct TcLayout {
     static constexpr int kThreads = 128 + 128 * NSLOT;
     static constexpr uint32_t kTmemCols = 512;
     // registers per thread after the split: warpgroup 0 gives, the softmax groups take
-    static constexpr uint32_t kRegsControl = 56;
-    static constexpr uint32_t kRegsSoftmax = 224;
+    static constexpr uint32_t kRegsControl = 40;
+    static constexpr uint32_t kRegsSoftmax = 232;
     static constexpr uint32_t kRegsNeeded = 128 * kRegsControl + 128 * NSLOT * kRegsSoftmax;
     static constexpr int kQ = 0;
     static constexpr int kKV = NSLOT * tc::kTileBytes;                 // [slot][stage] K + V^T

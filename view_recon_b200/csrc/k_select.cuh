@@ -27,8 +27,8 @@
 #define SEL_MAX_WARPS 8
 #define SEL_H1 1024        // first level: key bits 31..22
 #define SEL_H2 256         // refinement digits: bits 21..14, 13..6, 5..0
-#define SEL_LCAP 1024      // boundary-bin keys gathered for refinement
-#define SEL_SMEM_BUDGET (200 * 1024)
+#define SEL_LCAP 256       // boundary-bin keys gathered for refinement (more: refined from the row)
+#define SEL_SMEM_BUDGET (44 * 1024)  // per CTA: small CTAs of few rows keep ~20 warps per SM resident
 
 struct SelectArgs {
     const float* scores;  // row (local y, local x) at scores + (y * rows + x) * lds
