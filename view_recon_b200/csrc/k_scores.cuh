@@ -2,10 +2,13 @@
 // candidate interactions per head).
 //
 // SIMT f32: the ranking must be exact to about 1e-6 relative, which rules out a single-pass
-// tf32/bf16 tensor-core product.  A 256-thread CTA computes a 64 x 64 block of one head with
-// both 64 x 64 operand blocks staged in shared memory; every thread owns a 4 x 4 sub-block
-// and accumulates the 64 products in ascending e with FMA.  Rows [i0, i0 + rows) of head
-// h0 + blockIdx.z are written at out + (blockIdx.z * rows + local row) * ldo.
+// tf32/bf16 tensor-core product.  Every output accumulates its 64 products in ascending e with
+// FMA.  Rows [i0, i0 + rows) of head h0 + blockIdx.z are written at
+// out + (blockIdx.z * rows + local row) * ldo.
+//   tile_scores_kernel      64 x 64 blocks, 4 x 4 per thread (small tile counts: more CTAs);
+//   tile_scores_big_kernel  128 x 128 blocks, 8 x 8 per thread, operands transposed in shared
+//                           memory so a thread reads its 8 + 8 operands as four 16-byte words,
+//                           packed f32x2 FMAs (large tile counts).
 #pragma once
 #include "sa_device.cuh"
 
@@ -61,6 +64,76 @@ __global__ void __launch_bounds__(256) tile_scores_kernel(ScoreArgs a) {
         for (int w = 0; w < 4; ++w) {
             const int c = c_blk + tx + 16 * w;
             if (c < a.nt) ob[(int64_t)r * a.ldo + c] = acc[u][w];
+        }
+    }
+}
+
+#define SCORES_BIG_SMEM (2 * 64 * 128 * 4)
+
+// 128 x 128 block per 256-thread CTA; dynamic shared memory SCORES_BIG_SMEM (qT, kT: [64][128]).
+__global__ void __launch_bounds__(256) tile_scores_big_kernel(ScoreArgs a) {
+    extern __shared__ __align__(16) float big_smem[];
+    float* qT = big_smem;             // [64 e][128 rows]
+    float* kT = big_smem + 64 * 128;  // [64 e][128 cols]
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int h = a.h0 + blockIdx.z;
+    const int r_blk = blockIdx.y * 128;
+    const int c_blk = blockIdx.x * 128;
+    const float* qb = a.q_pool + ((int64_t)h * a.nt + a.i0) * 64;
+    const float* kb = a.k_pool + (int64_t)h * a.nt * 64;
+    // consecutive lanes take consecutive rows, so the transposed shared-memory writes of a warp
+    // fall into 32 different banks
+    for (int idx = threadIdx.x; idx < 128 * 16; idx += 256) {
+        const int r = idx & 127, c4 = idx >> 7;  // row r, elements 4 c4 .. 4 c4 + 3
+        float4 x = make_float4(0, 0, 0, 0), y = x;
+        if (r_blk + r < a.rows) x = __ldg(reinterpret_cast<const float4*>(qb + (int64_t)(r_blk + r) * 64) + c4);
+        if (c_blk + r < a.nt) y = __ldg(reinterpret_cast<const float4*>(kb + (int64_t)(c_blk + r) * 64) + c4);
+        qT[(4 * c4 + 0) * 128 + r] = x.x;
+        qT[(4 * c4 + 1) * 128 + r] = x.y;
+        qT[(4 * c4 + 2) * 128 + r] = x.z;
+        qT[(4 * c4 + 3) * 128 + r] = x.w;
+        kT[(4 * c4 + 0) * 128 + r] = y.x;
+        kT[(4 * c4 + 1) * 128 + r] = y.y;
+        kT[(4 * c4 + 2) * 128 + r] = y.z;
+        kT[(4 * c4 + 3) * 128 + r] = y.w;
+    }
+    __syncthreads();
+    float2 acc[8][4];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) acc[u][p] = make_float2(0.f, 0.f);
+#pragma unroll 4
+    for (int e = 0; e < 64; ++e) {
+        const float4 qa = *reinterpret_cast<const float4*>(qT + e * 128 + ty * 8);
+        const float4 qc = *reinterpret_cast<const float4*>(qT + e * 128 + ty * 8 + 4);
+        const float4 ka = *reinterpret_cast<const float4*>(kT + e * 128 + tx * 8);
+        const float4 kc = *reinterpret_cast<const float4*>(kT + e * 128 + tx * 8 + 4);
+        const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qc.x, qc.y, qc.z, qc.w};
+        const float2 kv[4] = {make_float2(ka.x, ka.y), make_float2(ka.z, ka.w), make_float2(kc.x, kc.y),
+                              make_float2(kc.z, kc.w)};
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int p = 0; p < 4; ++p) acc[u][p] = __ffma2_rn(make_float2(qv[u], qv[u]), kv[p], acc[u][p]);
+    }
+    float* ob = a.out + (int64_t)blockIdx.z * a.rows * a.ldo;
+    const int c0 = c_blk + tx * 8;
+    const bool vec = ((a.ldo & 3) == 0) && (c0 + 8 <= a.nt);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int r = r_blk + ty * 8 + u;
+        if (r >= a.rows) continue;
+        float* dst = ob + (int64_t)r * a.ldo + c0;
+        if (vec) {
+            reinterpret_cast<float4*>(dst)[0] = make_float4(acc[u][0].x, acc[u][0].y, acc[u][1].x, acc[u][1].y);
+            reinterpret_cast<float4*>(dst)[1] = make_float4(acc[u][2].x, acc[u][2].y, acc[u][3].x, acc[u][3].y);
+        } else {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                if (c0 + 2 * p < a.nt) dst[2 * p] = acc[u][p].x;
+                if (c0 + 2 * p + 1 < a.nt) dst[2 * p + 1] = acc[u][p].y;
+            }
         }
     }
 }

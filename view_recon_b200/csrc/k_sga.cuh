@@ -7,8 +7,8 @@
 // On the device this is three steps around the dense tensor-core attention:
 //   sga_gather_kernel   compacts the kept K/V rows of every frame into one key sequence of
 //                       S * (n_special + ceil(grid_h/s_h) * ceil(grid_w/s_w)) rows per head and
-//                       sums each frame's discarded K/V rows in fp32;
-//   sga_sum_kernel      adds the per-frame sums into one sum per head (fixed order);
+//                       sums the discarded K/V rows of each quarter frame in fp32;
+//   sga_sum_kernel      adds the partial sums into one sum per head (fixed order);
 //   (attention)         every query over the compacted keys: O and the natural-log LSE;
 //   sga_combine_kernel  per query row, folds in the diagonal (for a query whose own token was
 //                       discarded) and the mean pair of the other discarded columns:
@@ -24,12 +24,14 @@ struct SgaGeo {
     int32_t kpf;     // kept tokens per frame: n_special + kh * kw
 };
 
+#define SGA_SPLIT 4  // CTAs per frame in the gather
+
 struct SgaGatherArgs {
     const uint32_t* k;  // [bh][L][32] bf16 pairs
     const uint32_t* v;
     uint32_t* ksub;     // [bh][Lk][32]
     uint32_t* vsub;
-    float* part;        // [bh][S][2][64] per-frame sums of the discarded K (0) and V (1) rows
+    float* part;        // [bh][S * SGA_SPLIT][2][64] partial sums of the discarded K (0) and V (1) rows
     int32_t L, Lk;
     SgaGeo g;
 };
@@ -38,15 +40,28 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) {
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
-// One CTA of 8 warps per (frame, head).  A token row (64 bf16) is one 4-byte word per lane.
+__device__ __forceinline__ void acc_bf16x8(float (&s)[16], int off, const uint4& w) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        s[off + 2 * i] += __uint_as_float(u[i] << 16);
+        s[off + 2 * i + 1] += __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+}
+
+// SGA_SPLIT CTAs of 8 warps per (frame, head); CTA q takes every SGA_SPLIT-th kept row and a
+// contiguous quarter of the frame's patch tokens.  For the discarded sums a warp covers 8
+// consecutive tokens per step: lane l reads elements [16 (l & 3), 16 (l & 3) + 16) of token
+// l >> 2 as two 16-byte words of K and two of V, so every lane keeps four loads in flight.
 __global__ void __launch_bounds__(256) sga_gather_kernel(SgaGatherArgs a) {
-    __shared__ float2 red[8][2][32];
+    __shared__ float red[8][2][64];
     const SgaGeo& g = a.g;
-    const int f = blockIdx.x, h = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int f = blockIdx.x, q = blockIdx.y, h = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row0 = (int64_t)h * a.L + (int64_t)f * g.tokens;
     const int64_t out0 = (int64_t)h * a.Lk + (int64_t)f * g.kpf;
     // kept rows: the special tokens, then the grid positions (r * s_h, c * s_w) row-major
-    for (int e = warp; e < g.kpf; e += 8) {
+    for (int e = q * 8 + warp; e < g.kpf; e += 8 * SGA_SPLIT) {
         int n = e;
         if (e >= g.n_special) {
             const int p = e - g.n_special, rr = p / g.kw, cc = p - rr * g.kw;
@@ -55,44 +70,61 @@ __global__ void __launch_bounds__(256) sga_gather_kernel(SgaGatherArgs a) {
         a.ksub[(out0 + e) * 32 + lane] = __ldg(a.k + (row0 + n) * 32 + lane);
         a.vsub[(out0 + e) * 32 + lane] = __ldg(a.v + (row0 + n) * 32 + lane);
     }
-    // discarded rows: warp w sums grid rows w, w + 8, ...
-    float2 sk = make_float2(0.f, 0.f), sv = make_float2(0.f, 0.f);
-    for (int r = warp; r < g.grid_h; r += 8) {
-        const bool row_on_grid = (r % g.s_h) == 0;
-        const int64_t t0 = row0 + g.n_special + (int64_t)r * g.grid_w;
-        int cm = 0;  // c mod s_w
-        for (int c = 0; c < g.grid_w; ++c) {
-            if (!(row_on_grid && cm == 0)) {
-                const float2 kv = bf16x2_to_f2(__ldg(a.k + (t0 + c) * 32 + lane));
-                const float2 vv = bf16x2_to_f2(__ldg(a.v + (t0 + c) * 32 + lane));
-                sk.x += kv.x;
-                sk.y += kv.y;
-                sv.x += vv.x;
-                sv.y += vv.y;
-            }
-            if (++cm == g.s_w) cm = 0;
+    // discarded rows of this CTA's quarter of the patch grid
+    const int np = g.grid_h * g.grid_w;
+    const int per = (np + SGA_SPLIT - 1) / SGA_SPLIT;
+    const int p_lo = q * per, p_hi = min(np, p_lo + per);
+    const int sub = lane >> 2, quarter = lane & 3;
+    float sk[16], sv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sk[i] = sv[i] = 0.f;
+    for (int p0 = p_lo + warp * 8; p0 < p_hi; p0 += 64) {
+        const int p = p0 + sub;
+        bool take = p < p_hi;
+        if (take) {
+            const int r = p / g.grid_w, c = p - r * g.grid_w;
+            take = !((r % g.s_h) == 0 && (c % g.s_w) == 0);
+        }
+        if (take) {
+            const uint4* kr = reinterpret_cast<const uint4*>(a.k + (row0 + g.n_special + p) * 32) + 2 * quarter;
+            const uint4* vr = reinterpret_cast<const uint4*>(a.v + (row0 + g.n_special + p) * 32) + 2 * quarter;
+            const uint4 k0 = __ldg(kr), k1 = __ldg(kr + 1), v0 = __ldg(vr), v1 = __ldg(vr + 1);
+            acc_bf16x8(sk, 0, k0);
+            acc_bf16x8(sk, 8, k1);
+            acc_bf16x8(sv, 0, v0);
+            acc_bf16x8(sv, 8, v1);
         }
     }
-    red[warp][0][lane] = sk;
-    red[warp][1][lane] = sv;
-    __syncthreads();
-    if (warp < 2) {
-        float2 s = make_float2(0.f, 0.f);
-        for (int w = 0; w < 8; ++w) {
-            s.x += red[w][warp][lane].x;
-            s.y += red[w][warp][lane].y;
+    // lanes with the same quarter hold partial sums of the same 16 elements
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], off);
+            sv[i] += __shfl_xor_sync(0xffffffffu, sv[i], off);
         }
-        float* dst = a.part + (((int64_t)h * g.frames + f) * 2 + warp) * 64;
-        dst[2 * lane] = s.x;
-        dst[2 * lane + 1] = s.y;
+    if (lane < 4) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            red[warp][0][16 * lane + i] = sk[i];
+            red[warp][1][16 * lane + i] = sv[i];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 128) {
+        const int kv = threadIdx.x >> 6, e = threadIdx.x & 63;
+        float t = 0.f;
+        for (int w = 0; w < 8; ++w) t += red[w][kv][e];
+        a.part[(((int64_t)h * g.frames + f) * SGA_SPLIT + q) * 128 + threadIdx.x] = t;
     }
 }
 
-// sums[h][0 or 1][64] = sum over frames of part[h][f][0 or 1][64]; one CTA of 128 threads per head.
-__global__ void __launch_bounds__(128) sga_sum_kernel(const float* part, float* sums, int32_t frames) {
+// sums[h][0 or 1][64] = sum over the S * SGA_SPLIT partial sums of head h, in a fixed order; one
+// CTA of 128 threads per head.
+__global__ void __launch_bounds__(128) sga_sum_kernel(const float* part, float* sums, int32_t parts) {
     const int h = blockIdx.x, i = threadIdx.x;  // i = kv * 64 + e
     float s = 0.f;
-    for (int f = 0; f < frames; ++f) s += part[((int64_t)h * frames + f) * 128 + i];
+    for (int f = 0; f < parts; ++f) s += part[((int64_t)h * parts + f) * 128 + i];
     sums[(int64_t)h * 128 + i] = s;
 }
 
@@ -116,54 +148,69 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-// One warp per query row.
+#define SGA_ROWS_PER_WARP 2
+
+__device__ __forceinline__ float half_sum(float x) {  // sum over the 16 lanes of a half-warp
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+__device__ __forceinline__ float4 bf16x4_to_f4(uint2 u) {
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                       __uint_as_float(u.y & 0xFFFF0000u));
+}
+
+// One half-warp per query row (two rows per warp, four elements per lane), so each warp
+// instruction serves two rows and a dot product needs four shuffles.
 __global__ void __launch_bounds__(256) sga_combine_kernel(SgaCombineArgs a) {
-    const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (row >= a.rows) return;
+    const int lane = threadIdx.x & 31, hl = lane & 15;
+    const int64_t row = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * 2 + (lane >> 4);
+    const bool valid = row < a.rows;
+    const int64_t rr = valid ? row : a.rows - 1;  // the tail's idle half mirrors the last row
     const SgaGeo& g = a.g;
-    const int h = (int)(row / a.L);
-    const int t = (int)(row - (int64_t)h * a.L);
+    const int h = (int)(rr / a.L);
+    const int t = (int)(rr - (int64_t)h * a.L);
     const int n = t % g.tokens;
     bool kept = n < g.n_special;
     if (!kept) {
         const int p = n - g.n_special, r = p / g.grid_w, c = p - r * g.grid_w;
         kept = (r % g.s_h) == 0 && (c % g.s_w) == 0;
     }
-    const float2 q2 = bf16x2_to_f2(__ldg(a.q + row * 32 + lane));
-    const float2 o2 = bf16x2_to_f2(a.o[row * 32 + lane]);
-    const float lse = a.lse_in[row];
-    const float* sk = a.sums + (int64_t)h * 128;
-    float2 km = make_float2(sk[2 * lane], sk[2 * lane + 1]);
-    float2 vm = make_float2(sk[64 + 2 * lane], sk[64 + 2 * lane + 1]);
-    float2 vt = make_float2(0.f, 0.f);
+    const uint2* q2p = reinterpret_cast<const uint2*>(a.q) + rr * 16 + hl;
+    uint2* o2p = reinterpret_cast<uint2*>(a.o) + rr * 16 + hl;
+    const float4 q4 = bf16x4_to_f4(__ldg(q2p));
+    const float4 o4 = bf16x4_to_f4(*o2p);
+    const float lse = a.lse_in[rr];
+    const float4* sk4 = reinterpret_cast<const float4*>(a.sums + (int64_t)h * 128);
+    float4 km = __ldg(sk4 + hl), vm = __ldg(sk4 + 16 + hl);
+    float4 vt = make_float4(0.f, 0.f, 0.f, 0.f);
     float a_d = -INFINITY;
     int cnt = a.n_disc;
     if (!kept) {  // the diagonal is kept on its own; the mean pair covers the other discarded columns
-        const float2 kt = bf16x2_to_f2(__ldg(a.k + row * 32 + lane));
-        vt = bf16x2_to_f2(__ldg(a.v + row * 32 + lane));
-        a_d = a.scale * warp_sum(q2.x * kt.x + q2.y * kt.y);
-        km.x -= kt.x;
-        km.y -= kt.y;
-        vm.x -= vt.x;
-        vm.y -= vt.y;
+        const float4 kt = bf16x4_to_f4(__ldg(reinterpret_cast<const uint2*>(a.k) + rr * 16 + hl));
+        vt = bf16x4_to_f4(__ldg(reinterpret_cast<const uint2*>(a.v) + rr * 16 + hl));
+        a_d = q4.x * kt.x + q4.y * kt.y + q4.z * kt.z + q4.w * kt.w;
+        km.x -= kt.x; km.y -= kt.y; km.z -= kt.z; km.w -= kt.w;
+        vm.x -= vt.x; vm.y -= vt.y; vm.z -= vt.z; vm.w -= vt.w;
         cnt -= 1;
     }
-    float a_m = -INFINITY;
-    if (cnt > 0) {
-        const float inv = 1.0f / (float)cnt;
-        km.x *= inv;
-        km.y *= inv;
-        vm.x *= inv;
-        vm.y *= inv;
-        a_m = a.scale * warp_sum(q2.x * km.x + q2.y * km.y) + logf((float)cnt);
-    }
-    const float mx = fmaxf(lse, fmaxf(a_d, a_m));
-    const float w0 = expf(lse - mx), wd = expf(a_d - mx), wm = expf(a_m - mx);
+    const float inv = cnt > 0 ? 1.0f / (float)cnt : 0.0f;
+    const float dm = (q4.x * km.x + q4.y * km.y + q4.z * km.z + q4.w * km.w) * inv;
+    // both half-warps reduce together (the two rows of a warp may differ in `kept`)
+    const float sd = half_sum(kept ? 0.0f : a_d);
+    const float sm = half_sum(dm);
+    const float ad = kept ? -INFINITY : a.scale * sd;
+    const float am = cnt > 0 ? a.scale * sm + logf((float)cnt) : -INFINITY;
+    const float mx = fmaxf(lse, fmaxf(ad, am));
+    const float w0 = expf(lse - mx), wd = expf(ad - mx), wm = expf(am - mx);
     const float tot = w0 + wd + wm;
-    const float inv_tot = 1.0f / tot;
-    const float ox = (w0 * o2.x + wd * vt.x + wm * vm.x) * inv_tot;
-    const float oy = (w0 * o2.y + wd * vt.y + wm * vm.y) * inv_tot;
-    a.o[row * 32 + lane] = pack_bf16x2(ox, oy);
-    if (a.lse_out && lane == 0) a.lse_out[row] = mx + logf(tot);
+    const float f0 = w0 / tot, fd = wd / tot, fm = wm * inv / tot;
+    if (valid) {
+        uint2 out;
+        out.x = pack_bf16x2(f0 * o4.x + fd * vt.x + fm * vm.x, f0 * o4.y + fd * vt.y + fm * vm.y);
+        out.y = pack_bf16x2(f0 * o4.z + fd * vt.z + fm * vm.z, f0 * o4.w + fd * vt.w + fm * vm.w);
+        *o2p = out;
+        if (a.lse_out && hl == 0) a.lse_out[row] = mx + logf(tot);
+    }
 }

@@ -101,6 +101,8 @@ sa_status ensure_attributes() {
                                200 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                200 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tile_scores_big_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SCORES_BIG_SMEM) == cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SEL_SMEM_BUDGET) == cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -484,6 +486,18 @@ sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, cons
     return launch_status();
 }
 
+// Large tile counts: 128 x 128 blocks (8 x 8 outputs per thread); small ones keep 64 x 64 blocks
+// so that enough CTAs fill the GPU.
+static void launch_scores(const ScoreArgs& a, unsigned gz, cudaStream_t stream) {
+    if (a.nt >= 1024 && a.rows >= 128) {
+        const dim3 grid((unsigned)((a.nt + 127) / 128), (unsigned)((a.rows + 127) / 128), gz);
+        tile_scores_big_kernel<<<grid, 256, SCORES_BIG_SMEM, stream>>>(a);
+    } else {
+        const dim3 grid((unsigned)((a.nt + 63) / 64), (unsigned)((a.rows + 63) / 64), gz);
+        tile_scores_kernel<<<grid, 256, 0, stream>>>(a);
+    }
+}
+
 sa_status sa_tile_scores(const sa_shape* shape, const float* q_pool, const float* k_pool, float* scores,
                          sa_stream_t stream) {
     Geo g;
@@ -501,9 +515,9 @@ sa_status sa_tile_scores(const sa_shape* shape, const float* q_pool, const float
     a.h0 = 0;
     a.i0 = 0;
     a.rows = (int32_t)g.nt;
-    const dim3 grid((unsigned)((g.nt + 63) / 64), (unsigned)((g.nt + 63) / 64), (unsigned)g.bh);
     if ((g.nt + 63) / 64 > 65535) return SA_ERR_UNSUPPORTED;
-    tile_scores_kernel<<<grid, 256, 0, stream>>>(a);
+    if ((st = ensure_attributes()) != SA_OK) return st;
+    launch_scores(a, (unsigned)g.bh, stream);
     return launch_status();
 }
 
@@ -584,8 +598,7 @@ static sa_status select_impl(const sa_shape* shape, const float* scores_or_null,
             sc.h0 = (int32_t)h;
             sc.i0 = (int32_t)i0;
             sc.rows = (int32_t)rows;
-            tile_scores_kernel<<<dim3((unsigned)((g.nt + 63) / 64), (unsigned)((rows + 63) / 64), 1), 256, 0,
-                                 stream>>>(sc);
+            launch_scores(sc, 1u, stream);
             if ((st = launch_status()) != SA_OK) return st;
             a.scores = blk;
             a.lds = g.nt;
@@ -653,8 +666,7 @@ sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, con
             sc.h0 = (int32_t)h;
             sc.i0 = (int32_t)i0;
             sc.rows = (int32_t)rows;
-            tile_scores_kernel<<<dim3((unsigned)((g.nt + 63) / 64), (unsigned)((rows + 63) / 64), 1), 256, 0,
-                                 stream>>>(sc);
+            launch_scores(sc, 1u, stream);
             if ((st = launch_status()) != SA_OK) return st;
             a.scores = blk;
             a.lds = g.nt;
@@ -760,7 +772,7 @@ static sa_status sga_plan(const Geo& g, int32_t grid_h, int32_t grid_w, int32_t 
     w->vsub = off;
     off += align256((size_t)g.bh * w->Lk * 128);
     w->part = off;
-    off += align256((size_t)g.bh * g.S * 128 * 4);
+    off += align256((size_t)g.bh * g.S * SGA_SPLIT * 128 * 4);
     w->sums = off;
     off += align256((size_t)g.bh * 128 * 4);
     w->lse = off;
@@ -807,10 +819,10 @@ sa_status sa_sga_fwd(const sa_shape* shape, int32_t grid_h, int32_t grid_w, int3
     ga.L = (int32_t)g.L;
     ga.Lk = (int32_t)w.Lk;
     ga.g = w.sg;
-    sga_gather_kernel<<<dim3((unsigned)g.S, (unsigned)g.bh), 256, 0, stream>>>(ga);
+    sga_gather_kernel<<<dim3((unsigned)g.S, SGA_SPLIT, (unsigned)g.bh), 256, 0, stream>>>(ga);
     if ((st = launch_status()) != SA_OK) return st;
     float* sums = reinterpret_cast<float*>(base + w.sums);
-    sga_sum_kernel<<<(unsigned)g.bh, 128, 0, stream>>>(ga.part, sums, (int32_t)g.S);
+    sga_sum_kernel<<<(unsigned)g.bh, 128, 0, stream>>>(ga.part, sums, (int32_t)(g.S * SGA_SPLIT));
     if ((st = launch_status()) != SA_OK) return st;
     float* lse_att = reinterpret_cast<float*>(base + w.lse);
     st = attn_common(g, q, ga.ksub, ga.vsub, nullptr, nullptr, 0, nullptr, nullptr, 0, nullptr, nullptr, nullptr,
@@ -829,7 +841,8 @@ sa_status sa_sga_fwd(const sa_shape* shape, int32_t grid_h, int32_t grid_w, int3
     ca.n_disc = (int32_t)w.n_disc;
     ca.scale = g.scale;
     ca.g = w.sg;
-    sga_combine_kernel<<<(unsigned)((ca.rows + 7) / 8), 256, 0, stream>>>(ca);
+    sga_combine_kernel<<<(unsigned)((ca.rows + 8 * SGA_ROWS_PER_WARP - 1) / (8 * SGA_ROWS_PER_WARP)), 256, 0,
+                         stream>>>(ca);
     return launch_status();
 }
 
