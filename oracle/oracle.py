@@ -301,6 +301,89 @@ def attend_bruteforce(g: Geometry, q, k, v, kept, scale: float, landmark: bool =
     return O, LSE
 
 
+# ----------------------------------------------------------------------------- backward of step 4
+
+def attend_backward(g: Geometry, q: np.ndarray, k: np.ndarray, v: np.ndarray, kept, do: np.ndarray,
+                    scale: float, landmark: bool = False, cnt: np.ndarray | None = None, items=None):
+    """Gradients (dq, dk, dv) of sum(do * O) for O = attend(g, q, k, v, kept, scale, landmark).
+
+    The kept lists are constants of the layer call: selection is piecewise constant in its
+    inputs, so no gradient flows through pooling and scoring into it.  The landmark tokens
+    are differentiable functions of K and V (the tile means), so their gradients flow back
+    to the tile's non-sink rows, each receiving 1/c_j of it ("Zebra3D", abstract: landmark
+    summaries of unselected tiles, used for post-conversion training).
+    Per query tile, with the attended keys and values stacked in the forward's order:
+      P  = softmax(logits)                 (the forward's probabilities)
+      dV_att += P^T dO,   dP = dO V_att^T, Dr = rowsum(dO * O)
+      dS = P * (dP - Dr),  dQ = scale dS K_att,  dK_att += scale dS^T Q.
+    `items` restricts the query tiles taken as in `attend` (the gradients then cover only
+    their contributions).
+    """
+    bh, L, d = q.shape
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    if landmark:
+        _, k_bar, v_bar, cnt_p, _, _ = pool(g, q, k, v)
+        cnt = cnt_p if cnt is None else cnt
+        dk_bar = np.zeros((bh, g.nt, d))
+        dv_bar = np.zeros((bh, g.nt, v.shape[2]))
+    todo = items if items is not None else [(h, i) for h in range(bh) for i in range(g.nt)]
+    for h, i in todo:
+        rows = g.tile_rows(i)
+        kr = np.concatenate([g.tile_key_rows(int(j)) for j in kept[h][i]] + [g.sink_rows()])
+        qh, doh = q[h, rows], do[h, rows]
+        keys, vals = k[h, kr], v[h, kr]
+        logits = scale * (qh @ keys.T)
+        lm = np.zeros((0,), np.int64)
+        if landmark:
+            listed = np.zeros((g.nt,), bool)
+            listed[np.asarray(kept[h][i], np.int64)] = True
+            lm = np.nonzero((~listed) & (cnt > 0))[0]
+            logits = np.concatenate([logits, scale * (qh @ k_bar[h, lm].T) + np.log(cnt[lm].astype(np.float64))],
+                                    axis=1)
+            keys = np.concatenate([keys, k_bar[h, lm]], axis=0)
+            vals = np.concatenate([vals, v_bar[h, lm]], axis=0)
+        m = logits.max(axis=1, keepdims=True)
+        w = np.exp(logits - m)
+        p = w / w.sum(axis=1, keepdims=True)
+        o = p @ vals
+        d_v = p.T @ doh
+        dp = doh @ vals.T
+        dr = (doh * o).sum(axis=1, keepdims=True)
+        ds = p * (dp - dr)
+        dq[h, rows] += scale * (ds @ keys)
+        d_k = scale * (ds.T @ qh)
+        n_rows = len(kr)
+        np.add.at(dk[h], kr, d_k[:n_rows])
+        np.add.at(dv[h], kr, d_v[:n_rows])
+        if len(lm):
+            dk_bar[h, lm] += d_k[n_rows:]
+            dv_bar[h, lm] += d_v[n_rows:]
+    if landmark:  # k_bar_j is the mean of the c_j non-sink rows of tile j
+        for j in range(g.nt):
+            rk = g.tile_key_rows(j)
+            if len(rk):
+                dk[:, rk] += dk_bar[:, j][:, None, :] / len(rk)
+                dv[:, rk] += dv_bar[:, j][:, None, :] / len(rk)
+    return dq, dk, dv
+
+
+def dense_backward(q, k, v, do, scale: float):
+    """Gradients of sum(do * O) for textbook dense attention (the sparsity-0 control)."""
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for h in range(q.shape[0]):
+        lg = scale * (q[h] @ k[h].T)
+        w = np.exp(lg - lg.max(axis=1, keepdims=True))
+        p = w / w.sum(axis=1, keepdims=True)
+        o = p @ v[h]
+        dv[h] = p.T @ do[h]
+        ds = p * (do[h] @ v[h].T - (do[h] * o).sum(axis=1, keepdims=True))
+        dq[h] = scale * (ds @ k[h])
+        dk[h] = scale * (ds.T @ q[h])
+    return dq, dk, dv
+
+
 # ----------------------------------------------------------------------------- subsampled global attention
 
 def sga_kept(frames: int, tokens: int, n_special: int, grid_h: int, grid_w: int, s_h: int, s_w: int):
@@ -323,7 +406,7 @@ def sga_kept(frames: int, tokens: int, n_special: int, grid_h: int, grid_w: int,
 
 
 def sga(q, k, v, frames: int, tokens: int, n_special: int, grid_h: int, grid_w: int, s_h: int, s_w: int,
-        scale: float):
+        scale: float, rows=None):
     """Subsampled global attention ("AVGGT", technical summary 2.B.2, SGA).
 
     Every query attends to the kept tokens (sga_kept), to its own key (the diagonal is
@@ -331,7 +414,8 @@ def sga(q, k, v, frames: int, tokens: int, n_special: int, grid_h: int, grid_w: 
     the mean key and mean value of the discarded tokens of all frames - for a query whose own
     token is discarded, all of them except itself, since its column is kept as the diagonal -
     with a logit bias of ln(count), so that the pair weighs as the columns it replaces (the
-    aggregated response of the discarded columns is kept).  Returns (O [bh][L][d], LSE [bh][L]).
+    aggregated response of the discarded columns is kept).  Returns (O [bh][L][d], LSE [bh][L]);
+    with `rows` (token indices) only those query rows are computed (the others stay zero).
     """
     bh, L, _ = q.shape
     kept = sga_kept(frames, tokens, n_special, grid_h, grid_w, s_h, s_w)
@@ -343,7 +427,7 @@ def sga(q, k, v, frames: int, tokens: int, n_special: int, grid_h: int, grid_w: 
     for h in range(bh):
         k_sum = k[h, disc].sum(axis=0)
         v_sum = v[h, disc].sum(axis=0)
-        for t in range(L):
+        for t in (range(L) if rows is None else rows):
             own_disc = not kept[t]
             keys = [k[h, kidx]]
             vals = [v[h, kidx]]

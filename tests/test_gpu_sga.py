@@ -58,3 +58,49 @@ def test_sga_matches_oracle(frames, ns, gh, gw, sh, sw, src):
     if sh == 1 and sw == 1:
         O_d, L_d = orc.dense(Q, K, V, 0.125)
         H.check_attention(H.from_device(layer.o), H.from_device(layer.lse), O_d, L_d)
+
+
+def _sga_rows(w, rng, stride, n_random=48):
+    """Query rows that reach every case of the layer: special tokens, kept and discarded
+    patches, the last patch of a frame, in the first, middle and last frame, plus random rows."""
+    g = int(round((w.tokens - w.n_sink) ** 0.5))
+    fixed = []
+    for f in (0, w.frames // 2, w.frames - 1):
+        base = f * w.tokens
+        fixed += [base, base + w.n_sink - 1,                       # special tokens
+                  base + w.n_sink,                                 # patch (0, 0): kept
+                  base + w.n_sink + 1,                             # patch (0, 1): discarded
+                  base + w.n_sink + stride * g + stride,           # kept, interior
+                  base + w.tokens - 1]                             # last patch of the frame
+    rand = rng.choice(w.L, size=n_random, replace=False).tolist()
+    return sorted(set(fixed + rand))
+
+
+@pytest.mark.parametrize("wname,stride", [("vggt_s16_n1374", 3), ("vggt_s16_n1374", 9),
+                                          ("vggt_s128_n1374", 3)])
+def test_sga_full_size_sampled_rows(wname, stride):
+    """The benchmark's SGA launch (every head of the workload, 37 x 37 patch grid) compared with
+    the oracle on sampled query rows of the first and last head."""
+    import torch
+    import synth
+    from view_recon_b200 import sa
+    from view_recon_b200.pipeline import SubsampledGlobalAttention
+    from synth.workloads import VGGT_S16, VGGT_S128
+    w = {"vggt_s16_n1374": VGGT_S16, "vggt_s128_n1374": VGGT_S128}[wname]
+    grid = int(round((w.tokens - w.n_sink) ** 0.5))
+    data = synth.generate(w)
+    q, k, v = (H.to_device(data[x], w.dtype) for x in ("q", "k", "v"))
+    layer = SubsampledGlobalAttention(w.heads, w.frames, w.tokens, (grid, grid), (stride, stride),
+                                      w.n_sink, w.dtype, w.head_dim)
+    layer.forward(q, k, v)
+    torch.cuda.synchronize()
+    assert sa.sa_check_device_error() == 0
+    rng = np.random.default_rng(stride * 1000 + w.frames)
+    rows = _sga_rows(w, rng, stride)
+    idx = torch.as_tensor(rows, device="cuda")
+    for h in (0, w.heads - 1):
+        Q, K, V = (orc.to_f64(data[x][h:h + 1]) for x in ("q", "k", "v"))
+        O_ref, L_ref = orc.sga(Q, K, V, w.frames, w.tokens, w.n_sink, grid, grid, stride, stride,
+                               0.125, rows=rows)
+        H.check_attention(H.from_device(layer.o[h, idx]), H.from_device(layer.lse[h, idx]),
+                          O_ref[0, rows], L_ref[0, rows])

@@ -32,6 +32,9 @@ PIN_TESTS = [
     lambda: pins.test_k0_is_frame_attention_plus_sinks(),
     lambda: pins.test_sga_kept_positions(),
     *[lambda a=a, b=b: pins.test_sga_exact_when_discarded_tokens_are_identical(a, b) for a, b in ((2, 2), (3, 2))],
+    lambda: pins.test_backward_all_tiles_is_dense(2),
+    lambda: pins.test_backward_landmarks_exact_when_tile_rows_are_identical(),
+    lambda: pins.test_backward_matches_finite_differences(True, 1, 1),
 ]
 
 
@@ -183,7 +186,58 @@ def key_rows_keep_sinks(self, j):
     return f * self.tokens + np.arange(lo, hi)
 
 
+def _backward_variant(drop_rowsum=False, share_whole=False, dk_unscaled=False, dq_from_values=False,
+                      drop_lm_bias=False):
+    def attend_backward(g, q, k, v, kept, do, scale, landmark=False, cnt=None, items=None):
+        bh, L, d = q.shape
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+        if landmark:
+            _, k_bar, v_bar, cnt, _, _ = orc.pool(g, q, k, v)
+            dk_bar, dv_bar = np.zeros((bh, g.nt, d)), np.zeros((bh, g.nt, d))
+        for h in range(bh):
+            for i in range(g.nt):
+                rows = g.tile_rows(i)
+                kr = np.concatenate([g.tile_key_rows(int(j)) for j in kept[h][i]] + [g.sink_rows()])
+                keys, vals = k[h, kr], v[h, kr]
+                logits = scale * (q[h, rows] @ keys.T)
+                lm = np.zeros((0,), np.int64)
+                if landmark:
+                    listed = np.zeros((g.nt,), bool)
+                    listed[np.asarray(kept[h][i], np.int64)] = True
+                    lm = np.nonzero((~listed) & (cnt > 0))[0]
+                    b = 0.0 if drop_lm_bias else np.log(cnt[lm].astype(float))
+                    logits = np.concatenate([logits, scale * (q[h, rows] @ k_bar[h, lm].T) + b], axis=1)
+                    keys = np.concatenate([keys, k_bar[h, lm]])
+                    vals = np.concatenate([vals, v_bar[h, lm]])
+                w = np.exp(logits - logits.max(axis=1, keepdims=True))
+                p = w / w.sum(axis=1, keepdims=True)
+                dr = 0.0 if drop_rowsum else (do[h, rows] * (p @ vals)).sum(axis=1, keepdims=True)
+                ds = p * (do[h, rows] @ vals.T - dr)
+                dq[h, rows] += scale * (ds @ (vals if dq_from_values else keys))
+                d_k = (1.0 if dk_unscaled else scale) * (ds.T @ q[h, rows])
+                d_v = p.T @ do[h, rows]
+                np.add.at(dk[h], kr, d_k[:len(kr)])
+                np.add.at(dv[h], kr, d_v[:len(kr)])
+                if len(lm):
+                    dk_bar[h, lm] += d_k[len(kr):]
+                    dv_bar[h, lm] += d_v[len(kr):]
+        if landmark:
+            for j in range(g.nt):
+                rk = g.tile_key_rows(j)
+                if len(rk):
+                    c = 1 if share_whole else len(rk)
+                    dk[:, rk] += dk_bar[:, j][:, None, :] / c
+                    dv[:, rk] += dv_bar[:, j][:, None, :] / c
+        return dq, dk, dv
+    return attend_backward
+
+
 MUTANTS = {
+    "bwd_rowsum_term_dropped": ("attend_backward", _backward_variant(drop_rowsum=True)),
+    "bwd_landmark_gradient_not_shared": ("attend_backward", _backward_variant(share_whole=True)),
+    "bwd_dk_unscaled": ("attend_backward", _backward_variant(dk_unscaled=True)),
+    "bwd_dq_from_values": ("attend_backward", _backward_variant(dq_from_values=True)),
+    "bwd_landmark_bias_dropped": ("attend_backward", _backward_variant(drop_lm_bias=True)),
     "pool_includes_sinks": ("pool", pool_with_sinks),
     "scores_transposed": ("scores", scores_transposed),
     "ties_to_higher_index": ("select_row", select_ties_high),

@@ -397,3 +397,106 @@ def test_sga_exact_when_discarded_tokens_are_identical(s_h, s_w):
     O, LSE = orc.sga(q, k, v, S, N, ns, gh, gw, s_h, s_w, 0.25)
     Od, Ld = orc.dense(q, k, v, 0.25)
     assert np.abs(O - Od).max() < 1e-12 and np.abs(LSE - Ld).max() < 1e-12
+
+
+def test_sga_row_subset_matches_full():
+    """Computing only some query rows changes nothing for those rows and leaves the rest zero."""
+    rng = np.random.default_rng(5)
+    S, ns, gh, gw = 2, 3, 4, 6
+    N = ns + gh * gw
+    q, k, v = (rng.standard_normal((2, S * N, 8)) for _ in range(3))
+    O, LSE = orc.sga(q, k, v, S, N, ns, gh, gw, 2, 3, 0.25)
+    rows = [0, 4, 17, N + 5, 2 * N - 1]
+    Os, Ls = orc.sga(q, k, v, S, N, ns, gh, gw, 2, 3, 0.25, rows=rows)
+    assert np.array_equal(Os[:, rows], O[:, rows]) and np.array_equal(Ls[:, rows], LSE[:, rows])
+    rest = np.setdiff1d(np.arange(S * N), rows)
+    assert not Os[:, rest].any() and not Ls[:, rest].any()
+
+
+# ----------------------------------------------------------------------------- backward of the attention
+
+def _loss(g, q, k, v, kept, do, scale, landmark):
+    """sum(do * O) of the forward, with the landmark means recomputed from the given k, v."""
+    qb, kb, vb, cnt, _, _ = orc.pool(g, q, k, v)
+    O, _ = orc.attend(g, q, k, v, kept, scale, landmark, kb, vb, cnt)
+    return float((do * O).sum())
+
+
+@pytest.mark.parametrize("landmark", [False, True])
+@pytest.mark.parametrize("n_sink,kk", [(0, 1), (1, 1), (2, 0)])
+def test_backward_matches_finite_differences(landmark, n_sink, kk):
+    """Central differences of the forward (which the pins above fix) over every input
+    coordinate; the kept lists are held fixed, as the backward treats them."""
+    g, q, k, v = _tiny_case(60 + n_sink, frames=3, tokens=5, tile=2, n_sink=n_sink, bh=1, d=3)
+    scale = 0.45
+    qb, kb, _, _, _, _ = orc.pool(g, q, k, v)
+    kept = orc.select(g, orc.scores(qb, kb), kk)
+    do = rnd(q.shape, 77)
+    dq, dk, dv = orc.attend_backward(g, q, k, v, kept, do, scale, landmark)
+    eps = 1e-5
+    for x, grad in ((q, dq), (k, dk), (v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            keep = x[idx]
+            x[idx] = keep + eps
+            lp = _loss(g, q, k, v, kept, do, scale, landmark)
+            x[idx] = keep - eps
+            lm = _loss(g, q, k, v, kept, do, scale, landmark)
+            x[idx] = keep
+            fd[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, fd, rtol=0, atol=1e-8)
+
+
+def test_dense_backward_matches_autograd():
+    import torch
+    rng = np.random.default_rng(8)
+    q, k, v, do = (rng.standard_normal((2, 11, 5)) for _ in range(4))
+    dq, dk, dv = orc.dense_backward(q, k, v, do, 0.3)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    o = torch.softmax(0.3 * tq @ tk.transpose(1, 2), dim=-1) @ tv
+    (o * torch.tensor(do)).sum().backward()
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("n_sink", [0, 2])
+def test_backward_all_tiles_is_dense(n_sink):
+    g, q, k, v = _tiny_case(70, frames=3, tokens=6, tile=4, n_sink=n_sink, bh=2, d=4)
+    kept = [[np.arange(g.nt) for _ in range(g.nt)] for _ in range(2)]
+    do = rnd(q.shape, 71)
+    got = orc.attend_backward(g, q, k, v, kept, do, 0.4)
+    want = orc.dense_backward(q, k, v, do, 0.4)
+    for a, b in zip(got, want):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_backward_landmarks_exact_when_tile_rows_are_identical():
+    """Every tile's non-sink K rows equal one vector and its V rows another: the landmark of
+    an unselected tile then stands exactly for its rows in the forward and in every gradient
+    (the ln(c_j) bias and the 1/c_j share of the mean's gradient), so the gradients are the
+    dense ones for any selection.  With only the K rows identical, dq and dv stay dense and
+    dk keeps the dense sum over each tile's rows (a landmark spreads its share evenly)."""
+    g = orc.Geometry(frames=4, tokens=7, tile=3, n_sink=1)  # counts 2, 3, 1 per frame
+    d = 3
+    rng = np.random.default_rng(9)
+    q = rng.standard_normal((1, g.L, d))
+    do = rng.standard_normal((1, g.L, d))
+    k = rng.standard_normal((1, g.L, d))
+    v = rng.standard_normal((1, g.L, d))
+    for j in range(g.nt):
+        k[0, g.tile_key_rows(j)] = rng.standard_normal(d)
+    qb, kb, _, _, _, _ = orc.pool(g, q, k, v)
+    kept = orc.select(g, orc.scores(qb, kb), 1)
+    dq, dk, dv = orc.attend_backward(g, q, k, v, kept, do, 0.6, landmark=True)
+    dq_d, dk_d, dv_d = orc.dense_backward(q, k, v, do, 0.6)
+    np.testing.assert_allclose(dq, dq_d, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv, dv_d, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk[0, g.sink_rows()], dk_d[0, g.sink_rows()], rtol=0, atol=1e-12)
+    for j in range(g.nt):
+        rk = g.tile_key_rows(j)
+        np.testing.assert_allclose(dk[0, rk].sum(axis=0), dk_d[0, rk].sum(axis=0), rtol=0, atol=1e-12)
+    for j in range(g.nt):
+        v[0, g.tile_key_rows(j)] = rng.standard_normal(d)
+    _, dk, _ = orc.attend_backward(g, q, k, v, kept, do, 0.6, landmark=True)
+    _, dk_d, _ = orc.dense_backward(q, k, v, do, 0.6)
+    np.testing.assert_allclose(dk, dk_d, rtol=0, atol=1e-12)
