@@ -549,6 +549,130 @@ def run_sga(args, w):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------------------ backward arm
+
+def run_backward(args, w):
+    """--backward: one training step of the sparse layer, forward (pool, score, select, attend)
+    then backward (sa_sparse_attn_bwd) against a fixed upstream gradient, through the same
+    timing contract; the roofline is the backward call's (all of its launches)."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from view_recon_b200 import sa
+    from view_recon_b200.pipeline import SparseGlobalAttention
+
+    rank, world, local = rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    sa.load()
+    w_job = w
+    heads_local, head0, seed, calls_here = shard_plan(args.shard, w.heads, world, rank, w.seed)
+    w = w.scaled(heads=heads_local)
+    host = synth.generate(w, seed=seed, head0=head0)
+
+    def pinned(a):
+        return torch.from_numpy(a).view(torch.bfloat16).pin_memory()
+
+    rng = np.random.default_rng(seed + 17)
+    g32 = rng.standard_normal((w.heads, w.L, w.head_dim)).astype(np.float32)
+    gb = g32.view(np.uint32)
+    hdo = pinned(((gb + 0x7FFF + ((gb >> 16) & 1)) >> 16).astype(np.uint16))
+    hq, hk, hv = pinned(host["q"]), pinned(host["k"]), pinned(host["v"])
+    q, k, v, d_o = hq.to(dev), hk.to(dev), hv.to(dev), hdo.to(dev)
+    layer = SparseGlobalAttention(w.heads, w.frames, w.tokens, w.k, w.tile, w.n_sink, w.dtype, w.landmark,
+                                  w.streamed, w.head_dim, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step_events():
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        layer.forward(q, k, v)
+        ev[1].record(stream)
+        layer.backward(q, k, v, d_o)
+        ev[2].record(stream)
+        return ev
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step_events()
+    torch.cuda.synchronize(dev)
+    status = sa.sa_check_device_error()
+    if status != 0:
+        raise RuntimeError("device error after warm-up: %s" % sa.status_string(status))
+    fwd_flops, _ = attention_work(layer, w)
+    bwd_flops = 2.5 * fwd_flops  # five products of 2*d per attended (row, key) pair against the forward's two
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    dist_barrier(dev)
+    torch.cuda.synchronize(dev)
+    evs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        evs.append(step_events())
+    torch.cuda.synchronize(dev)
+    dist_barrier(dev)
+    clk = clocks.stop()
+    st_ms = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in evs])
+    total_ms = float(st_ms.sum())
+    max_total_ms = dist_max(total_ms, dev)
+    status = sa.sa_check_device_error()
+    if status != 0:
+        raise RuntimeError("device error in timed region: %s" % sa.status_string(status))
+    ms_fwd, ms_bwd = (float(x) for x in st_ms.mean(axis=0))
+    # end to end: Q, K, V and dO in from pinned host memory, dQ, dK, dV out, every step
+    hg = [torch.empty_like(hq).pin_memory() for _ in range(3)]
+    e2e_steps = max(3, min(args.steps, 10))
+    dist_barrier(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for dst, src in ((q, hq), (k, hk), (v, hv), (d_o, hdo)):
+            dst.copy_(src, non_blocking=True)
+        layer.forward(q, k, v)
+        grads = layer.backward(q, k, v, d_o)
+        for dst, src in zip(hg, grads):
+            dst.copy_(src, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = dist_max(e0.elapsed_time(e1), dev)
+    peaks, peak_src = measured_peaks()
+    achieved = bwd_flops / (ms_bwd / 1e3) / 1e12
+    nbytes = w.heads * w.L * w.head_dim * 2
+    line = {
+        "metric": "sparse global-attention training tokens/s (forward + backward)",
+        "value": whole_job_rate(w.L * calls_here, world, args.steps, max_total_ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak" if not (args.shard == "heads" and world > 1) else "strong",
+        "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic latent-point Q/K/V and upstream gradient (seeded; no dataset or weights)",
+        "config": {"workload": w_job.name + "_fwd_bwd", "frames": w.frames, "tokens_per_frame": w.tokens,
+                   "heads": w_job.heads, "head_dim": w.head_dim, "tile": w.tile, "n_sink": w.n_sink, "k": w.k,
+                   "landmark": w.landmark, "l2": "flushed before every step"},
+        "stages_ms": {"forward": ms_fwd, "backward": ms_bwd},
+        "bwd_tflops_algorithmic": achieved,
+        "roofline": {"bound": "tensor", "kernel": "sa_sparse_attn_bwd (all launches of the call)",
+                     "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "peak_source": "%s bf16 burst" % peak_src,
+                     "traffic": None, "algorithmic_flops_per_launch": bwd_flops},
+        "e2e": {"value": whole_job_rate(w.L * calls_here, world, e2e_steps, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 3 * nbytes},
+        "gpu_launches": (layer.launches_per_call() + layer.backward_launches()) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del layer
+    if world > 1:
+        dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------------------ the reference arm
 
 def run_reference(args, w):
@@ -590,6 +714,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sga", type=int, default=0, metavar="STRIDE",
                     help="time the AVGGT subsampled global attention layer (stride x stride grid) instead")
+    ap.add_argument("--backward", action="store_true",
+                    help="time a training step of the sparse layer (forward + backward) instead")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="with N > 1: independent layer call per GPU, or one layer call split by heads")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
@@ -602,6 +728,8 @@ def main(argv=None):
         run_reference(args, w)
     elif args.sga:
         run_sga(args, w)
+    elif args.backward:
+        run_backward(args, w)
     else:
         run_ours(args, w)
 

@@ -219,6 +219,42 @@ sa_status sa_sparse_attn_fwd(const sa_shape* shape, const void* q, const void* k
                              void* workspace_or_null, size_t workspace_bytes,
                              void* o, float* lse_or_null, sa_stream_t stream);
 
+/* Bytes of workspace sa_sparse_attn_bwd needs for these lists and mode (bf16, tile 128 only;
+ * 0 otherwise): transposed tiles of Q, dO and K, fp32 accumulators of dK and dV, the reverse
+ * lists and, in landmark mode, the landmark tables - roughly 8x the size of Q. */
+size_t sa_sparse_attn_bwd_workspace_size(const sa_shape* shape, int32_t max_kept, int32_t landmark);
+
+/*
+ * Backward of step 4, for training a backbone whose global layers are made sparse after
+ * conversion (Zebra3D abstract: tile-sparse attention with landmark summaries).
+ *
+ * Gradients of sum(d_o * O) for O = sa_sparse_attn_fwd(q, k, v, lists, ...), the lists held
+ * fixed (selection is piecewise constant in its inputs, so no gradient flows into it).  With
+ * P the forward's probabilities over each row's attended set and D_r = sum_e d_o[r][e] o[r][e]:
+ *   dS = P * (d_o V^T - D),  dq = scale dS K,  dk = scale dS^T Q,  dv = P^T d_o,
+ * summed over every query row that attends a key; a sink row receives its sink-segment terms;
+ * in landmark mode the landmark of tile j (the mean of its k_cnt[j] non-sink rows) passes its
+ * gradient to each of those rows divided by k_cnt[j].
+ *   q, k, v, o    the forward's inputs and output, [bh][S*N][64] bf16
+ *   lse           the forward's lse (natural log), f32 [bh][S*N]; required
+ *   d_o           upstream gradient, [bh][S*N][64] bf16
+ *   lists, sinks, landmark, pools: exactly as passed to sa_sparse_attn_fwd
+ *   dq, dk, dv    outputs, [bh][S*N][64] bf16, written in full (caller-owned, 16-byte aligned)
+ * Products run on the tensor cores (bf16 operands, f32 accumulation; P and dS enter rounded to
+ * bf16).  dk and dv are accumulated with f32 atomics, so the last bits of their values may
+ * vary between calls.  bf16, d = 64, tile = 128 only (else SA_ERR_UNSUPPORTED).  Bad list
+ * entries are skipped and reported as SA_ERR_BAD_LIST by sa_check_device_error.
+ * workspace: >= sa_sparse_attn_bwd_workspace_size(shape, max_kept, landmark) bytes.
+ */
+sa_status sa_sparse_attn_bwd(const sa_shape* shape, const void* q, const void* k, const void* v,
+                             const void* o, const float* lse, const void* d_o,
+                             const int32_t* kept_idx, const int32_t* kept_cnt, int32_t max_kept,
+                             const void* sink_k_or_null, const void* sink_v_or_null,
+                             int32_t landmark, const float* k_pool_or_null,
+                             const float* v_pool_or_null, const int32_t* k_cnt_or_null,
+                             void* workspace, size_t workspace_bytes,
+                             void* dq, void* dk, void* dv, sa_stream_t stream);
+
 /* Bytes of workspace sa_dense_attn_fwd needs (a transposed copy of V on the tensor-core
  * path, 0 on the CUDA-core path). */
 size_t sa_dense_attn_workspace_size(const sa_shape* shape);

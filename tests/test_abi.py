@@ -128,3 +128,34 @@ def test_sga_host_checks(lib):
     assert lib.sa_sga_fwd(s, 37, 37, 3, 3, fake, fake, fake, fake, 16, fake, None, None) == sa.SA_ERR_WORKSPACE
     assert lib.sa_sga_fwd(ctypes.byref(f32), 37, 37, 3, 3, fake, fake, fake, fake, 1 << 40, fake, None,
                           None) == sa.SA_ERR_UNSUPPORTED
+
+
+def test_backward_host_checks(lib):
+    from view_recon_b200 import sa
+    s = ctypes.byref(sa.shape(2, 3, 300, 64, 128, 5, "bf16"))
+    fake = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    args = lambda **kw: [kw.get(n, fake) for n in ("q", "k", "v", "o", "lse", "do")]  # noqa: E731
+    tail = lambda ws=1 << 40: [fake, fake, 0, None, None, None, fake, ws, fake, fake, fake, None]  # noqa: E731
+    need = sa.sa_sparse_attn_bwd_workspace_size(sa.shape(2, 3, 300, 64, 128, 5, "bf16"), 5, False)
+    assert need > 0
+    assert lib.sa_sparse_attn_bwd(s, *args(lse=None), fake, fake, 5, *tail()) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_sparse_attn_bwd(s, *args(o=odd), fake, fake, 5, *tail()) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_sparse_attn_bwd(s, *args(), fake, fake, 0, *tail()) == sa.SA_ERR_INVALID_ARG  # max_kept
+    assert lib.sa_sparse_attn_bwd(s, *args(), fake, fake, 5, *tail(ws=need - 1)) == sa.SA_ERR_WORKSPACE
+    # sinks missing while the shape has some
+    t = tail()
+    t[0] = None
+    assert lib.sa_sparse_attn_bwd(s, *args(), fake, fake, 5, *t) == sa.SA_ERR_INVALID_ARG
+    # landmark mode without the pools
+    t = tail()
+    t[2] = 1
+    assert lib.sa_sparse_attn_bwd(s, *args(), fake, fake, 5, *t) == sa.SA_ERR_INVALID_ARG
+    # f32 or tile 64: no backward
+    f32 = sa.shape(2, 3, 300, 64, 128, 5, "f32")
+    assert sa.sa_sparse_attn_bwd_workspace_size(f32, 5, False) == 0
+    assert lib.sa_sparse_attn_bwd(ctypes.byref(f32), *args(), fake, fake, 5, *tail()) == sa.SA_ERR_UNSUPPORTED
+    # the workspace grows with the lists and with landmarks
+    shp = sa.shape(16, 16, 1374, 64, 128, 5, "bf16")
+    assert sa.sa_sparse_attn_bwd_workspace_size(shp, 46, True) > sa.sa_sparse_attn_bwd_workspace_size(shp, 46, False)
+    assert sa.sa_sparse_attn_bwd_workspace_size(shp, 100, False) > sa.sa_sparse_attn_bwd_workspace_size(shp, 46, False)

@@ -5,6 +5,7 @@
 #include <mutex>
 #include <string.h>
 
+#include "k_attn_bwd.cuh"
 #include "k_attn_prep.cuh"
 #include "k_attn_simt.cuh"
 #include "k_attn_tc.cuh"
@@ -101,6 +102,10 @@ sa_status ensure_attributes() {
                                200 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                200 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)bw::QLay::smem_bytes()) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)bw::KVLay::smem_bytes()) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tile_scores_big_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SCORES_BIG_SMEM) == cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -844,6 +849,271 @@ sa_status sa_sga_fwd(const sa_shape* shape, int32_t grid_h, int32_t grid_w, int3
     sga_combine_kernel<<<(unsigned)((ca.rows + 8 * SGA_ROWS_PER_WARP - 1) / (8 * SGA_ROWS_PER_WARP)), 256, 0,
                          stream>>>(ca);
     return launch_status();
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ backward of the sparse attention
+
+namespace {
+
+// Workspace of the backward (offsets 256-byte aligned):
+//   lse2t, dt   per query tile row: LSE in base 2 and rowsum(dO*O)      f32 [bh][nt][128] each
+//   qt, dot, kt transposed tiles of Q, dO (query tiles) and K (key tiles) bf16 [bh][nt][64][128]
+//   skt         transposed sink K tiles                                   bf16 [bh][n_sink_tiles][64][128]
+//   lk, lv      landmark K / V rows, lkt transposed landmark K chunks,
+//               lvt scratch of the landmark table writer, lbias [ntp]     (landmark mode)
+//   bits        listed-tile bitmap of every query tile                    u32 [bh][nt][ntp/32] (landmark)
+//   rev_cnt, fill, rev, units, n_units   reverse lists and the dK/dV work units
+//   dk32, dv32  fp32 accumulators [bh][L][64]; dkbar, dvbar landmark gradients [bh][ntp][64]
+struct BwdWs {
+    int64_t ntp, n_sink_tiles, n_lm_chunks, words, units_cap;
+    size_t lse2t, dt, qt, dot, kt, skt, lk, lv, lkt, lvt, lbias, bits, rev_cnt, fill, rev, units, n_units, dk32,
+        dv32, dkbar, dvbar, total;
+};
+
+BwdWs bwd_ws(const Geo& g, int64_t max_kept, bool landmark) {
+    BwdWs w;
+    constexpr size_t kTile = 64 * 128 * 2;
+    w.ntp = (g.nt + 127) / 128 * 128;
+    w.n_sink_tiles = (g.S * g.n_sink + 127) / 128;
+    w.n_lm_chunks = landmark ? w.ntp / 128 : 0;
+    w.words = w.ntp / 32;
+    const int64_t chunks_q = (g.nt + kBwdChunk - 1) / kBwdChunk;
+    const int64_t M = g.bh * g.nt;
+    w.units_cap = g.bh * (w.n_sink_tiles + w.n_lm_chunks) * chunks_q + (M * max_kept) / kBwdChunk + M + 1;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += align256(bytes);
+        return at;
+    };
+    w.lse2t = take((size_t)M * 128 * 4);
+    w.dt = take((size_t)M * 128 * 4);
+    w.qt = take((size_t)M * kTile);
+    w.dot = take((size_t)M * kTile);
+    w.kt = take((size_t)M * kTile);
+    w.skt = take((size_t)g.bh * w.n_sink_tiles * kTile);
+    w.lk = take(landmark ? (size_t)g.bh * w.ntp * 128 : 0);
+    w.lv = take(landmark ? (size_t)g.bh * w.ntp * 128 : 0);
+    w.lkt = take((size_t)g.bh * w.n_lm_chunks * kTile);
+    w.lvt = take((size_t)g.bh * w.n_lm_chunks * kTile);
+    w.lbias = take(landmark ? (size_t)w.ntp * 4 : 0);
+    w.bits = take(landmark ? (size_t)M * w.words * 4 : 0);
+    w.rev_cnt = take((size_t)M * 4);
+    w.fill = take((size_t)M * 4);
+    w.rev = take((size_t)M * max_kept * 4);
+    w.units = take((size_t)w.units_cap * 16);
+    w.n_units = take(16);
+    w.dk32 = take((size_t)g.bh * g.L * 64 * 4);
+    w.dv32 = take((size_t)g.bh * g.L * 64 * 4);
+    w.dkbar = take(landmark ? (size_t)g.bh * w.ntp * 64 * 4 : 0);
+    w.dvbar = take(landmark ? (size_t)g.bh * w.ntp * 64 * 4 : 0);
+    w.total = off;
+    return w;
+}
+
+sa_status transpose_tiles(const void* src, void* dst, int64_t tiles_per_head, bool frame_mode, const Geo& g,
+                          int64_t rows_per_head, cudaStream_t stream) {
+    if (tiles_per_head < 1) return SA_OK;
+    VtArgs t;
+    t.src = static_cast<const __nv_bfloat16*>(src);
+    t.dst = static_cast<__nv_bfloat16*>(dst);
+    t.tiles_per_head = (int32_t)tiles_per_head;
+    t.frame_mode = frame_mode ? 1 : 0;
+    t.tokens = (int32_t)g.N;
+    t.tpf = (int32_t)g.tpf;
+    t.L = (int32_t)g.L;
+    t.rows_per_head = (int32_t)rows_per_head;
+    vtile_transpose_kernel<<<dim3((unsigned)tiles_per_head, (unsigned)g.bh), 256, 0, stream>>>(t);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sa_sparse_attn_bwd_workspace_size(const sa_shape* shape, int32_t max_kept, int32_t landmark) {
+    Geo g;
+    if (geo_of(shape, &g) != SA_OK || !use_tc(g)) return 0;
+    if (max_kept < 1 || max_kept > g.nt) return 0;
+    return bwd_ws(g, max_kept, landmark != 0).total;
+}
+
+sa_status sa_sparse_attn_bwd(const sa_shape* shape, const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* d_o, const int32_t* kept_idx, const int32_t* kept_cnt,
+                             int32_t max_kept, const void* sink_k_or_null, const void* sink_v_or_null,
+                             int32_t landmark, const float* k_pool_or_null, const float* v_pool_or_null,
+                             const int32_t* k_cnt_or_null, void* workspace, size_t workspace_bytes, void* dq, void* dk,
+                             void* dv, sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    const void* must[] = {q, k, v, o, lse, d_o, kept_idx, kept_cnt, dq, dk, dv};
+    for (const void* p : must)
+        if (!p || !aligned16(p)) return SA_ERR_INVALID_ARG;
+    if (max_kept < 1 || max_kept > g.nt) return SA_ERR_INVALID_ARG;
+    if (g.n_sink > 0 && (!sink_k_or_null || !sink_v_or_null || !aligned16(sink_k_or_null) ||
+                         !aligned16(sink_v_or_null)))
+        return SA_ERR_INVALID_ARG;
+    if (landmark && (!k_pool_or_null || !v_pool_or_null || !k_cnt_or_null || !aligned16(k_pool_or_null) ||
+                     !aligned16(v_pool_or_null) || !aligned16(k_cnt_or_null)))
+        return SA_ERR_INVALID_ARG;
+    if (!use_tc(g)) return SA_ERR_UNSUPPORTED;
+    const bool lm = landmark != 0;
+    const BwdWs w = bwd_ws(g, max_kept, lm);
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return SA_ERR_WORKSPACE;
+    if (g.bh > 65535 || g.bh * g.nt * max_kept >= (1ll << 31) || w.units_cap >= (1ll << 31) ||
+        g.nt >= (1 << 24) || g.bh * g.nt * 64 >= (1ll << 31))
+        return SA_ERR_UNSUPPORTED;
+    if ((st = ensure_attributes()) != SA_OK) return st;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    const int64_t M = g.bh * g.nt;
+    const int64_t n_sink_rows = g.S * g.n_sink;
+
+    BwdArgs a;
+    memset(&a, 0, sizeof(a));
+    TcArgs& t = a.geo;
+    bool ok = encode_rows_bf16(&t.tm_q, q, g.bh * g.L) && encode_rows_bf16(&t.tm_k, k, g.bh * g.L) &&
+              encode_vt_tiles(&t.tm_vt, base + w.kt, M) && encode_rows_bf16(&a.tm_do, d_o, g.bh * g.L) &&
+              encode_rows_bf16(&a.tm_v, v, g.bh * g.L) && encode_vt_tiles(&a.tm_qt, base + w.qt, M) &&
+              encode_vt_tiles(&a.tm_dot, base + w.dot, M);
+    if (w.n_sink_tiles > 0)
+        ok = ok && encode_rows_bf16(&t.tm_sk, sink_k_or_null, g.bh * n_sink_rows) &&
+             encode_rows_bf16(&a.tm_sv, sink_v_or_null, g.bh * n_sink_rows) &&
+             encode_vt_tiles(&t.tm_svt, base + w.skt, g.bh * w.n_sink_tiles);
+    else
+        t.tm_sk = t.tm_k, a.tm_sv = a.tm_v, t.tm_svt = t.tm_vt;
+    if (lm)
+        ok = ok && encode_rows_bf16(&t.tm_lk, base + w.lk, g.bh * w.ntp) &&
+             encode_rows_bf16(&a.tm_lv, base + w.lv, g.bh * w.ntp) &&
+             encode_vt_tiles(&t.tm_lvt, base + w.lkt, g.bh * w.n_lm_chunks);
+    else
+        t.tm_lk = t.tm_k, a.tm_lv = a.tm_v, t.tm_lvt = t.tm_vt;
+    if (!ok) return SA_ERR_CUDA;
+
+    // ---- per-row terms and transposed operand tiles
+    {
+        const int64_t rows = M * 128;
+        bwd_rows_kernel<<<(unsigned)((rows + 31) / 32), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), lse,
+            reinterpret_cast<float*>(base + w.lse2t), reinterpret_cast<float*>(base + w.dt), (int32_t)g.bh,
+            (int32_t)g.nt, (int32_t)g.tpf, (int32_t)g.N, (int32_t)g.L);
+        if ((st = launch_status()) != SA_OK) return st;
+    }
+    if ((st = transpose_tiles(q, base + w.qt, g.nt, true, g, g.L, stream)) != SA_OK) return st;
+    if ((st = transpose_tiles(d_o, base + w.dot, g.nt, true, g, g.L, stream)) != SA_OK) return st;
+    if ((st = transpose_tiles(k, base + w.kt, g.nt, true, g, g.L, stream)) != SA_OK) return st;
+    if (w.n_sink_tiles > 0 &&
+        (st = transpose_tiles(sink_k_or_null, base + w.skt, w.n_sink_tiles, false, g, n_sink_rows, stream)) != SA_OK)
+        return st;
+    if (lm) {
+        const int64_t n4 = g.bh * w.ntp * 16;
+        const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 148 * 32);
+        float* lbias = reinterpret_cast<float*>(base + w.lbias);
+        __nv_bfloat16* lvt = reinterpret_cast<__nv_bfloat16*>(base + w.lvt);
+        landmark_prep_kernel<<<blocks, 256, 0, stream>>>(k_pool_or_null, v_pool_or_null, k_cnt_or_null,
+                                                         reinterpret_cast<__nv_bfloat16*>(base + w.lk), lvt, lbias,
+                                                         (int32_t)g.bh, (int32_t)g.nt, (int32_t)w.ntp);
+        if ((st = launch_status()) != SA_OK) return st;
+        landmark_prep_kernel<<<blocks, 256, 0, stream>>>(v_pool_or_null, v_pool_or_null, k_cnt_or_null,
+                                                         reinterpret_cast<__nv_bfloat16*>(base + w.lv), lvt, lbias,
+                                                         (int32_t)g.bh, (int32_t)g.nt, (int32_t)w.ntp);
+        if ((st = launch_status()) != SA_OK) return st;
+        if ((st = transpose_tiles(base + w.lk, base + w.lkt, w.n_lm_chunks, false, g, w.ntp, stream)) != SA_OK)
+            return st;
+        if (cudaMemsetAsync(base + w.bits, 0, (size_t)M * w.words * 4, stream) != cudaSuccess) return SA_ERR_CUDA;
+    }
+
+    // ---- reverse lists and the dK/dV work units
+    int32_t* rev_cnt = reinterpret_cast<int32_t*>(base + w.rev_cnt);
+    int32_t* fill = reinterpret_cast<int32_t*>(base + w.fill);
+    if (cudaMemsetAsync(rev_cnt, 0, (size_t)M * 4, stream) != cudaSuccess) return SA_ERR_CUDA;
+    {
+        const int64_t total = M * max_kept;
+        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, (int64_t)sms * 16));
+        bwd_scan_lists_kernel<<<blocks, 256, 0, stream>>>(kept_idx, kept_cnt, max_kept, (int32_t)g.bh, (int32_t)g.nt,
+                                                          (int32_t)w.words,
+                                                          lm ? reinterpret_cast<uint32_t*>(base + w.bits) : nullptr,
+                                                          rev_cnt);
+        if ((st = launch_status()) != SA_OK) return st;
+        bwd_plan_kernel<<<1, 1024, 0, stream>>>(rev_cnt, fill, reinterpret_cast<int4*>(base + w.units),
+                                                reinterpret_cast<int32_t*>(base + w.n_units), (int32_t)g.bh,
+                                                (int32_t)g.nt, (int32_t)w.n_sink_tiles, (int32_t)w.n_lm_chunks);
+        if ((st = launch_status()) != SA_OK) return st;
+        bwd_fill_lists_kernel<<<blocks, 256, 0, stream>>>(kept_idx, kept_cnt, max_kept, (int32_t)g.bh, (int32_t)g.nt,
+                                                          fill, reinterpret_cast<int32_t*>(base + w.rev));
+        if ((st = launch_status()) != SA_OK) return st;
+    }
+    if (cudaMemsetAsync(base + w.dk32, 0, (size_t)g.bh * g.L * 64 * 4, stream) != cudaSuccess ||
+        cudaMemsetAsync(base + w.dv32, 0, (size_t)g.bh * g.L * 64 * 4, stream) != cudaSuccess)
+        return SA_ERR_CUDA;
+    if (lm && (cudaMemsetAsync(base + w.dkbar, 0, (size_t)g.bh * w.ntp * 64 * 4, stream) != cudaSuccess ||
+               cudaMemsetAsync(base + w.dvbar, 0, (size_t)g.bh * w.ntp * 64 * 4, stream) != cudaSuccess))
+        return SA_ERR_CUDA;
+
+    // ---- the two tensor-core kernels
+    t.kept_idx = kept_idx;
+    t.kept_cnt = kept_cnt;
+    t.lbias2 = lm ? reinterpret_cast<const float*>(base + w.lbias) : nullptr;
+    t.max_kept = max_kept;
+    t.frames = (int32_t)g.S;
+    t.tokens = (int32_t)g.N;
+    t.n_sink = (int32_t)g.n_sink;
+    t.tpf = (int32_t)g.tpf;
+    t.nt = (int32_t)g.nt;
+    t.L = (int32_t)g.L;
+    t.Lk = (int32_t)g.L;
+    t.ntp = (int32_t)w.ntp;
+    t.n_vtiles = (int32_t)g.nt;
+    t.n_sink_rows = (int32_t)n_sink_rows;
+    t.n_sink_tiles = (int32_t)w.n_sink_tiles;
+    t.n_lm_chunks = (int32_t)w.n_lm_chunks;
+    t.dense = 0;
+    t.landmark = lm ? 1 : 0;
+    t.q_per_head = (int32_t)g.nt;
+    t.total_items = (int32_t)M;
+    t.scale_log2 = (float)((double)g.scale * 1.4426950408889634);
+    t.tpf_magic = 0;
+    if (g.tpf > 1) {
+        t.tpf_magic = (uint32_t)((0x100000000ull + (uint64_t)g.tpf - 1) / (uint64_t)g.tpf);
+        for (int64_t j = 0; j < g.nt; ++j)
+            if ((int64_t)(((uint64_t)j * t.tpf_magic) >> 32) != j / g.tpf) return SA_ERR_UNSUPPORTED;
+    }
+    a.lse2t = reinterpret_cast<const float*>(base + w.lse2t);
+    a.dt = reinterpret_cast<const float*>(base + w.dt);
+    a.listed_bits = lm ? reinterpret_cast<const uint32_t*>(base + w.bits) : nullptr;
+    a.units = reinterpret_cast<const int4*>(base + w.units);
+    a.n_units = reinterpret_cast<const int32_t*>(base + w.n_units);
+    a.rev = reinterpret_cast<const int32_t*>(base + w.rev);
+    a.dq = static_cast<__nv_bfloat16*>(dq);
+    a.dk32 = reinterpret_cast<float*>(base + w.dk32);
+    a.dv32 = reinterpret_cast<float*>(base + w.dv32);
+    a.dkbar = lm ? reinterpret_cast<float*>(base + w.dkbar) : nullptr;
+    a.dvbar = lm ? reinterpret_cast<float*>(base + w.dvbar) : nullptr;
+    a.scale = g.scale;
+    attn_bwd_dq_kernel<<<(unsigned)M, bw::kThreads, bw::QLay::smem_bytes(), stream>>>(a);
+    if ((st = launch_status()) != SA_OK) return st;
+    const int grid = (int)std::min<int64_t>(sms, w.units_cap);
+    attn_bwd_dkv_kernel<<<grid, bw::kThreads, bw::KVLay::smem_bytes(), stream>>>(a);
+    if ((st = launch_status()) != SA_OK) return st;
+    {
+        const int64_t total = g.bh * g.L * 8;
+        const int blocks = (int)std::min<int64_t>((total + 255) / 256, (int64_t)sms * 32);
+        bwd_finalize_kernel<<<blocks, 256, 0, stream>>>(
+            reinterpret_cast<const float*>(base + w.dk32), reinterpret_cast<const float*>(base + w.dv32),
+            lm ? reinterpret_cast<const float*>(base + w.dkbar) : nullptr,
+            lm ? reinterpret_cast<const float*>(base + w.dvbar) : nullptr, static_cast<__nv_bfloat16*>(dk),
+            static_cast<__nv_bfloat16*>(dv), (int32_t)g.bh, (int32_t)g.L, (int32_t)g.N, (int32_t)g.tpf,
+            (int32_t)g.n_sink, (int32_t)w.ntp);
+        if ((st = launch_status()) != SA_OK) return st;
+    }
+    return SA_OK;
 }
 
 }  // extern "C"

@@ -34,6 +34,14 @@ class Buffers:
     lse: object
 
 
+@dataclasses.dataclass
+class GradBuffers:
+    ws: object
+    dq: object
+    dk: object
+    dv: object
+
+
 class SparseGlobalAttention:
     """Dynamic tile-sparse global attention for bh heads of S frames x N tokens (d = 64).
 
@@ -89,6 +97,7 @@ class SparseGlobalAttention:
             o=torch.empty((bh, self.L, head_dim), dtype=tdt, device=dev),
             lse=torch.empty((bh, self.L), dtype=f32, device=dev) if with_lse else None,
         )
+        self.grad = None  # backward buffers, allocated by the first backward call
 
     # individual steps (each one C call) ---------------------------------------------------------
     def pool(self, q, k, v, stream=None):
@@ -122,6 +131,39 @@ class SparseGlobalAttention:
         return self.buf.o, self.buf.lse
 
     __call__ = forward
+
+    def backward(self, q, k, v, d_o, stream=None):
+        """Gradients (dq, dk, dv) of sum(d_o * O) for the last forward on these q, k, v, with its
+        kept lists held fixed; d_o is [bh][S*N][d] like O.  Needs the forward's LSE."""
+        import torch
+        b = self.buf
+        if b.lse is None:
+            raise ValueError("the backward needs the forward's LSE (with_lse=True)")
+        if self.grad is None:
+            nbytes = sa.sa_sparse_attn_bwd_workspace_size(self.shape, self.max_kept, self.landmark)
+            if nbytes == 0:
+                raise ValueError("no backward for this shape (bf16, tile 128, d 64 only)")
+            dev = self.device
+            self.grad = GradBuffers(
+                ws=torch.empty((nbytes,), dtype=torch.uint8, device=dev),
+                dq=torch.empty((self.bh, self.L, self.d), dtype=self.dtype, device=dev),
+                dk=torch.empty((self.bh, self.L, self.d), dtype=self.dtype, device=dev),
+                dv=torch.empty((self.bh, self.L, self.d), dtype=self.dtype, device=dev),
+            )
+        gr = self.grad
+        sa.sa_sparse_attn_bwd(self.shape, q, k, v, b.o, b.lse, d_o, b.kept_idx, b.kept_cnt, self.max_kept,
+                              b.sink_k, b.sink_v, self.landmark, b.k_pool, b.v_pool, b.k_cnt, gr.ws, gr.dq, gr.dk,
+                              gr.dv, stream)
+        return gr.dq, gr.dk, gr.dv
+
+    def backward_launches(self) -> int:
+        """Kernel launches libsa makes for one backward (memsets not counted)."""
+        n = 1 + 3 + 3 + 3  # row terms; Q, dO, K transposes; list scan, plan, fill; dQ, dK/dV, finalize
+        if self.frames * self.shape.n_sink > 0:
+            n += 1  # transposed sink K tiles
+        if self.landmark:
+            n += 3  # landmark K and V tables, transposed landmark K chunks
+        return n
 
     def launches_per_call(self) -> int:
         """Kernel launches libsa makes for one forward (for launch accounting)."""

@@ -29,7 +29,8 @@ SA_BF16 = 1
 EXPORTS = [
     "sa_num_tiles", "sa_max_kept", "sa_tile_pool", "sa_tile_scores", "sa_select_workspace_size",
     "sa_select_topk", "sa_select_topk_per_head", "sa_select_topk_noalloc", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
-    "sa_dense_attn_fwd", "sa_sga_workspace_size", "sa_sga_fwd",
+    "sa_dense_attn_fwd", "sa_sga_workspace_size", "sa_sga_fwd", "sa_sparse_attn_bwd_workspace_size",
+    "sa_sparse_attn_bwd",
     "sa_status_string", "sa_check_device_error", "sa_set_wait_limit_ns", "sa_test_withhold_query_load",
 ]
 
@@ -87,6 +88,9 @@ def load(path: str | None = None):
         "sa_sga_workspace_size": (sz, [shp, i32, i32, i32, i32]),
         "sa_sga_fwd": (i32, [shp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp, vp]),
         "sa_test_withhold_query_load": (i32, [i32]),
+        "sa_sparse_attn_bwd_workspace_size": (sz, [shp, i32, i32]),
+        "sa_sparse_attn_bwd": (i32, [shp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp,
+                                     vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -203,6 +207,20 @@ def sa_dense_attn_fwd(shp, q, k, v, workspace, o, lse=None, stream=None):
     st = load().sa_dense_attn_fwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(workspace), ws_bytes, _ptr(o),
                                   _ptr(lse), _stream(stream))
     _check("sa_dense_attn_fwd", st)
+
+
+def sa_sparse_attn_bwd_workspace_size(shp, max_kept, landmark=False) -> int:
+    return int(load().sa_sparse_attn_bwd_workspace_size(ctypes.byref(shp), int(max_kept), 1 if landmark else 0))
+
+
+def sa_sparse_attn_bwd(shp, q, k, v, o, lse, d_o, kept_idx, kept_cnt, max_kept, sink_k, sink_v, landmark, k_pool,
+                       v_pool, k_cnt, workspace, dq, dk, dv, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().sa_sparse_attn_bwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(d_o),
+                                   _ptr(kept_idx), _ptr(kept_cnt), int(max_kept), _ptr(sink_k), _ptr(sink_v),
+                                   1 if landmark else 0, _ptr(k_pool), _ptr(v_pool), _ptr(k_cnt), _ptr(workspace),
+                                   ws_bytes, _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream))
+    _check("sa_sparse_attn_bwd", st)
 
 
 def sa_check_device_error(stream=None) -> int:
