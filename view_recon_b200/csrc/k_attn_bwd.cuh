@@ -57,14 +57,20 @@ struct __align__(64) BwdArgs {
 namespace bw {
 
 constexpr int kT = tc::kTileBytes;
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;   // warps 0-3 control, warpgroups 1-4 the elementwise work
+constexpr int kCompute = 512;
 
+// Operands come through two rings per kernel, each with its own producer warp: the row tiles
+// read by the S / dP products (released as soon as those complete) and the transposed tiles
+// read by the gradient products (released after them), so that the next tiles' copies start
+// early and their latency stays off the tensor pipe's path.
 struct QLay {
-    static constexpr int STAGES = 3;
-    static constexpr int kQ = 0, kDO = kT, kRing = 2 * kT;
-    static constexpr int kStage = 3 * kT;  // K rows, V rows, K^T
-    static constexpr int kBars = kRing + STAGES * kStage;
-    static constexpr int kNumBars = 1 + 2 * STAGES + 5;
+    static constexpr int RS = 4, TS = 3;
+    static constexpr int kQ = 0, kDO = kT;
+    static constexpr int kRows = 2 * kT, kRowStage = 2 * kT;  // [RS] K rows, V rows
+    static constexpr int kTr = kRows + RS * kRowStage, kTrStage = kT;  // [TS] K^T
+    static constexpr int kBars = kTr + TS * kTrStage;
+    static constexpr int kNumBars = 1 + 2 * RS + 2 * TS + 5;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kEnd = kMisc + 16;
     static constexpr uint32_t colS = 0, colDP = 128, colDS = 256, colDQ = 320;
@@ -72,11 +78,12 @@ struct QLay {
 };
 
 struct KVLay {
-    static constexpr int STAGES = 2;
-    static constexpr int kK = 0, kV = kT, kRing = 2 * kT;
-    static constexpr int kStage = 4 * kT + 1024;  // Q rows, dO rows, Q^T, dO^T, lse2[128], D[128]
-    static constexpr int kBars = kRing + STAGES * kStage;
-    static constexpr int kNumBars = 2 * STAGES + 11;
+    static constexpr int RS = 3, TS = 2;
+    static constexpr int kK = 0, kV = kT;
+    static constexpr int kRows = 2 * kT, kRowStage = 2 * kT;                  // [RS] Q rows, dO rows
+    static constexpr int kTr = kRows + RS * kRowStage, kTrStage = 2 * kT + 1024;  // [TS] Q^T, dO^T, lse2, D
+    static constexpr int kBars = kTr + TS * kTrStage;
+    static constexpr int kNumBars = 2 * RS + 2 * TS + 9;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kEnd = kMisc + 16;
     static constexpr uint32_t colS = 0, colDP = 128, colP = 256, colDS = 320, colDV = 384, colDK = 448;
@@ -99,9 +106,9 @@ __device__ __forceinline__ void query_tile(const TcArgs& g, int h, int i, int32_
 
 // ------------------------------------------------------------------------------ dQ
 
-__global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
     using Lay = bw::QLay;
-    constexpr int STAGES = Lay::STAGES;
+    constexpr int RS = Lay::RS, TS = Lay::TS;
     constexpr int kT = bw::kT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = bw::align1024(smem_raw);
@@ -110,12 +117,15 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* sQ = smem + Lay::kQ;
     uint8_t* sDO = smem + Lay::kDO;
-    uint8_t* sRing = smem + Lay::kRing;
+    uint8_t* sRows = smem + Lay::kRows;
+    uint8_t* sTr = smem + Lay::kTr;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBars);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = kv_full + STAGES;
-    uint64_t* sd_full = kv_empty + STAGES;
+    uint64_t* rows_full = bars + 1;
+    uint64_t* rows_empty = rows_full + RS;
+    uint64_t* t_full = rows_empty + RS;
+    uint64_t* t_empty = t_full + TS;
+    uint64_t* sd_full = t_empty + TS;
     uint64_t* sd_free = sd_full + 1;
     uint64_t* ds_full = sd_free + 1;
     uint64_t* dq_done = ds_full + 1;
@@ -124,13 +134,17 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+        for (int s = 0; s < RS; ++s) {
+            mbar_init(&rows_full[s], 1);
+            mbar_init(&rows_empty[s], 1);
+        }
+        for (int s = 0; s < TS; ++s) {
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], 1);
         }
         mbar_init(sd_full, 1);
-        mbar_init(sd_free, 256);
-        mbar_init(ds_full, 256);
+        mbar_init(sd_free, bw::kCompute);
+        mbar_init(ds_full, bw::kCompute);
         mbar_init(dq_done, 1);
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -147,41 +161,51 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
     const tc::Slot sl = tc::make_slot(g, blockIdx.x);
     const int n_items = sl.n_items;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------------------------ TMA producers
+        // warp 0: Q, dO, then K and V rows of every item; warp 2: the transposed K tiles
+        const bool rows = warp == 0;
+        const int depth = rows ? RS : TS;
+        uint64_t* full = rows ? rows_full : t_full;
+        uint64_t* empty = rows ? rows_empty : t_empty;
         const bool leader = tc::elect_one();
         uint32_t issued_mask = 0, phase_mask = 0;
         bool ok = true;
-        if (n_items > 0 && leader) {
+        if (rows && n_items > 0 && leader) {
             mbar_arrive_expect_tx(q_full, 2 * kT);
             tma_load_2d(sQ, &g.tm_q, q_full, 0, sl.qrow);
             tma_load_2d(sDO, &a.tm_do, q_full, 0, sl.qrow);
         }
         for (int n = 0; n < n_items; ++n) {
-            const uint32_t s = n % STAGES, ph = (n / STAGES) & 1u;
-            if (!mbar_wait_warp(&kv_empty[s], ph ^ 1u, abort_flag)) {
+            const uint32_t s = n % depth, ph = (n / depth) & 1u;
+            if (!mbar_wait_warp(&empty[s], ph ^ 1u, abort_flag)) {
                 ok = false;
                 break;
             }
             if (leader) {
                 const tc::Item it = tc::get_item(g, sl, n);
-                const CUtensorMap* mk = it.kind == 1 ? &g.tm_sk : (it.kind == 2 ? &g.tm_lk : &g.tm_k);
-                const CUtensorMap* mv = it.kind == 1 ? &a.tm_sv : (it.kind == 2 ? &a.tm_lv : &a.tm_v);
-                const CUtensorMap* mt = it.kind == 1 ? &g.tm_svt : (it.kind == 2 ? &g.tm_lvt : &g.tm_vt);
-                uint8_t* d = sRing + s * Lay::kStage;
-                mbar_arrive_expect_tx(&kv_full[s], 3 * kT);
-                tma_load_2d(d, mk, &kv_full[s], 0, it.krow);
-                tma_load_2d(d + kT, mv, &kv_full[s], 0, it.krow);
-                tma_load_2d(d + 2 * kT, mt, &kv_full[s], 0, it.vrow);
-                tma_load_2d(d + 2 * kT + kT / 2, mt, &kv_full[s], 64, it.vrow);
+                if (rows) {
+                    const CUtensorMap* mk = it.kind == 1 ? &g.tm_sk : (it.kind == 2 ? &g.tm_lk : &g.tm_k);
+                    const CUtensorMap* mv = it.kind == 1 ? &a.tm_sv : (it.kind == 2 ? &a.tm_lv : &a.tm_v);
+                    uint8_t* d = sRows + s * Lay::kRowStage;
+                    mbar_arrive_expect_tx(&full[s], 2 * kT);
+                    tma_load_2d(d, mk, &full[s], 0, it.krow);
+                    tma_load_2d(d + kT, mv, &full[s], 0, it.krow);
+                } else {
+                    const CUtensorMap* mt = it.kind == 1 ? &g.tm_svt : (it.kind == 2 ? &g.tm_lvt : &g.tm_vt);
+                    uint8_t* d = sTr + s * Lay::kTrStage;
+                    mbar_arrive_expect_tx(&full[s], kT);
+                    tma_load_2d(d, mt, &full[s], 0, it.vrow);
+                    tma_load_2d(d + kT / 2, mt, &full[s], 64, it.vrow);
+                }
             }
             issued_mask |= 1u << s;
             phase_mask = (phase_mask & ~(1u << s)) | (ph << s);
         }
         if (!ok) {
-            for (int s = 0; s < STAGES; ++s)
-                if ((issued_mask >> s) & 1u) tc::drain_wait(&kv_full[s], (phase_mask >> s) & 1u);
-            if (n_items > 0) tc::drain_wait(q_full, 0);
+            for (int s = 0; s < depth; ++s)
+                if ((issued_mask >> s) & 1u) tc::drain_wait(&full[s], (phase_mask >> s) & 1u);
+            if (rows && n_items > 0) tc::drain_wait(q_full, 0);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
@@ -191,42 +215,45 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
         tc_fence_after();
         const uint64_t dq_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
         const uint64_t ddo = smem_desc_sw128(smem_u32(sDO), 16, 1024);
-        const uint64_t dk0 = smem_desc_sw128(smem_u32(sRing), 16, 1024);
-        const uint64_t dv0 = smem_desc_sw128(smem_u32(sRing + kT), 16, 1024);
-        const uint64_t dt0 = smem_desc_sw128(smem_u32(sRing + 2 * kT), 16, 1024);
-        constexpr uint64_t kStep = (uint64_t)Lay::kStage >> 4;
+        const uint64_t dk0 = smem_desc_sw128(smem_u32(sRows), 16, 1024);
+        const uint64_t dv0 = smem_desc_sw128(smem_u32(sRows + kT), 16, 1024);
+        const uint64_t dt0 = smem_desc_sw128(smem_u32(sTr), 16, 1024);
+        constexpr uint64_t kRowStep = (uint64_t)Lay::kRowStage >> 4;
+        constexpr uint64_t kTrStep = (uint64_t)Lay::kTrStage >> 4;
         for (int n = 0; n <= n_items && ok; ++n) {
             if (n < n_items) {
-                const uint32_t s = n % STAGES, ph = (n / STAGES) & 1u;
-                if (!mbar_wait_warp(&kv_full[s], ph, abort_flag)) { ok = false; break; }
+                const uint32_t s = n % RS, ph = (n / RS) & 1u;
+                if (!mbar_wait_warp(&rows_full[s], ph, abort_flag)) { ok = false; break; }
                 if (n > 0 && !mbar_wait_warp(sd_free, (n - 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 if (leader) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_ss(tmem + Lay::colS, dq_desc + 2 * kk, dk0 + s * kStep + 2 * kk, tc::kIdescS, kk > 0);
+                        umma_ss(tmem + Lay::colS, dq_desc + 2 * kk, dk0 + s * kRowStep + 2 * kk, tc::kIdescS, kk > 0);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_ss(tmem + Lay::colDP, ddo + 2 * kk, dv0 + s * kStep + 2 * kk, tc::kIdescS, kk > 0);
+                        umma_ss(tmem + Lay::colDP, ddo + 2 * kk, dv0 + s * kRowStep + 2 * kk, tc::kIdescS, kk > 0);
                     umma_commit(sd_full);
+                    umma_commit(&rows_empty[s]);
                 }
                 __syncwarp();
                 any_mma = true;
             }
             if (n >= 1) {
                 const int m = n - 1;
-                const uint32_t s = m % STAGES;
+                const uint32_t s = m % TS, ph = (m / TS) & 1u;
                 if (!mbar_wait_warp(ds_full, m & 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait_warp(&t_full[s], ph, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 if (leader) {
-                    const uint64_t dt = dt0 + s * kStep;
+                    const uint64_t dt = dt0 + s * kTrStep;
                     // K^T is two 64-key swizzle atoms of 8 KB; a K=16 step is 32 bytes
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         umma_ts(tmem + Lay::colDQ, tmem + Lay::colDS + 8 * kk,
                                 dt + (uint64_t)((kk >> 2) * (8192 >> 4) + (kk & 3) * 2), tc::kIdescPV,
                                 (m > 0 || kk > 0));
-                    umma_commit(&kv_empty[s]);
+                    umma_commit(&t_empty[s]);
                     umma_commit(dq_done);
                 }
                 __syncwarp();
@@ -239,20 +266,23 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------------ dS (thread = query row)
-        const int hc = (warp - 4) >> 2;  // key columns [64 hc, 64 hc + 64)
+        const int hc = (warp - 4) >> 2;  // key columns [32 hc, 32 hc + 32)
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t tS = tmem + Lay::colS + lane_off + hc * 64;
-        const uint32_t tDP = tmem + Lay::colDP + lane_off + hc * 64;
-        const uint32_t tDS = tmem + Lay::colDS + lane_off + hc * 32;
-        const uint32_t tDQ = tmem + Lay::colDQ + lane_off + hc * 32;
+        const uint32_t tS = tmem + Lay::colS + lane_off + hc * 32;
+        const uint32_t tDP = tmem + Lay::colDP + lane_off + hc * 32;
+        const uint32_t tDS = tmem + Lay::colDS + lane_off + hc * 16;
+        const uint32_t tDQ = tmem + Lay::colDQ + lane_off + hc * 16;
         float lse2 = INFINITY, drow = 0.0f;
         if (sl.active) {
             const int64_t ti = ((int64_t)sl.h * g.nt + sl.i) * 128 + r;
             lse2 = __ldg(a.lse2t + ti);
             drow = __ldg(a.dt + ti);
         }
+        const float2 scale2 = make_float2(g.scale_log2, g.scale_log2);
+        const float2 nl2 = make_float2(-lse2, -lse2);
+        const float2 nd2 = make_float2(-drow, -drow);
         bool ok = true;
         int lm_ptr = 0;
         for (int n = 0; n < n_items; ++n) {
@@ -271,25 +301,40 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
             }
             if (!mbar_wait_warp(sd_full, n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            uint32_t pk[32];
+            uint32_t sv[32], dp[32];
+            tmem_ld_32x32b_x32(tS, sv);
+            tmem_ld_32x32b_x32(tDP, dp);
+            tmem_ld_wait(sv);
+            reg_fence(dp);
+            tc_fence_before();
+            mbar_arrive(sd_free);  // the next item's products may overwrite S and dP now
+            uint32_t pk[16];
+            const int c0 = hc * 32;
+            if (it.kind >= 0 && it.kind <= 1 && it.lo == 0 && it.hi == 128) {
+                // whole tile attended: no mask, no bias
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t sv[32], dp[32];
-                tmem_ld_32x32b_x32(tS + half * 32, sv);
-                tmem_ld_32x32b_x32(tDP + half * 32, dp);
-                tmem_ld_wait(sv);
-                reg_fence(dp);
-                if (half == 1) {
-                    tc_fence_before();
-                    mbar_arrive(sd_free);
+                for (int u = 0; u < 16; ++u) {
+                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * u]), __uint_as_float(sv[2 * u + 1])),
+                                                scale2, nl2);
+                    float2 p;
+                    if ((u & 7) >= 8 - SA_EXP2_FMA_PAIRS_PER8) {
+                        p = exp2_poly2(x);
+                    } else {
+                        p.x = ex2_approx(x.x);
+                        p.y = ex2_approx(x.y);
+                    }
+                    const float2 d = __fmul2_rn(
+                        p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * u]), __uint_as_float(dp[2 * u + 1])), nd2));
+                    pk[u] = pack_bf16x2(d.x, d.y);
                 }
-                const int c0 = hc * 64 + half * 32;
+            } else {
+                // partial tile, sink chunk tail, landmark chunk or skipped entry: per-column terms
 #pragma unroll
-                for (int u = 0; u < 32; u += 2) {
-                    float ds2[2];
+                for (int u = 0; u < 16; ++u) {
+                    float d2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int c = c0 + u + e;
+                        const int c = c0 + 2 * u + e;
                         bool valid;
                         float b = 0.0f;
                         if (it.kind == 2) {
@@ -298,31 +343,31 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
                         } else {
                             valid = c >= it.lo && c < it.hi;
                         }
-                        const float x = fmaf(__uint_as_float(sv[u + e]), g.scale_log2, b) - lse2;
+                        const float x = fmaf(__uint_as_float(sv[2 * u + e]), g.scale_log2, b) - lse2;
                         const float p = valid ? ex2_approx(x) : 0.0f;
-                        ds2[e] = p * (__uint_as_float(dp[u + e]) - drow);
+                        d2[e] = p * (__uint_as_float(dp[2 * u + e]) - drow);
                     }
-                    pk[half * 16 + u / 2] = pack_bf16x2(ds2[0], ds2[1]);
+                    pk[u] = pack_bf16x2(d2[0], d2[1]);
                 }
             }
             if (n > 0) {
                 if (!mbar_wait_warp(dq_done, (n - 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
             }
-            tmem_st_32x32b_x32(tDS, pk);
+            tmem_st_32x32b_x16(tDS, pk);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(ds_full);
         }
         if (ok && n_items > 0 && mbar_wait_warp(dq_done, (n_items - 1) & 1, abort_flag)) {
             tc_fence_after();
-            uint32_t acc[32];
-            tmem_ld_32x32b_x32(tDQ, acc);
-            tmem_ld_wait(acc);
+            uint32_t acc[16];
+            tmem_ld_32x32b_x16(tDQ, acc);
+            tmem_ld_wait16(acc);
             if (r < sl.nq) {
-                uint4* dst = reinterpret_cast<uint4*>(a.dq + ((int64_t)sl.qrow + r) * 64 + hc * 32);
+                uint4* dst = reinterpret_cast<uint4*>(a.dq + ((int64_t)sl.qrow + r) * 64 + hc * 16);
 #pragma unroll
-                for (int c8 = 0; c8 < 4; ++c8) {
+                for (int c8 = 0; c8 < 2; ++c8) {
                     uint4 w;
                     w.x = pack_bf16x2(__uint_as_float(acc[8 * c8 + 0]) * a.scale, __uint_as_float(acc[8 * c8 + 1]) * a.scale);
                     w.y = pack_bf16x2(__uint_as_float(acc[8 * c8 + 2]) * a.scale, __uint_as_float(acc[8 * c8 + 3]) * a.scale);
@@ -332,9 +377,9 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dq_kernel(const __grid_consta
                 }
             }
         } else if (ok && sl.active && n_items == 0 && r < sl.nq) {
-            uint4* dst = reinterpret_cast<uint4*>(a.dq + ((int64_t)sl.qrow + r) * 64 + hc * 32);
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) dst[c8] = make_uint4(0, 0, 0, 0);
+            uint4* dst = reinterpret_cast<uint4*>(a.dq + ((int64_t)sl.qrow + r) * 64 + hc * 16);
+            dst[0] = make_uint4(0, 0, 0, 0);
+            dst[1] = make_uint4(0, 0, 0, 0);
         }
     }
 
@@ -392,9 +437,9 @@ __device__ __forceinline__ int unit_query_tile(const BwdArgs& a, const Unit& x, 
 
 }  // namespace bw
 
-__global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_constant__ BwdArgs a) {
+__global__ void __launch_bounds__(640, 1) attn_bwd_dkv_kernel(const __grid_constant__ BwdArgs a) {
     using Lay = bw::KVLay;
-    constexpr int STAGES = Lay::STAGES;
+    constexpr int RS = Lay::RS, TS = Lay::TS;
     constexpr int kT = bw::kT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = bw::align1024(smem_raw);
@@ -403,11 +448,14 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* sK = smem + Lay::kK;
     uint8_t* sV = smem + Lay::kV;
-    uint8_t* sRing = smem + Lay::kRing;
+    uint8_t* sRows = smem + Lay::kRows;
+    uint8_t* sTr = smem + Lay::kTr;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBars);
-    uint64_t* st_fullb = bars;                // [STAGES] stage loaded
-    uint64_t* st_empty = bars + STAGES;       // [STAGES] stage consumed
-    uint64_t* kvu_full = bars + 2 * STAGES;   // unit's K, V rows loaded
+    uint64_t* rows_full = bars;               // [RS] Q, dO rows of a pair loaded
+    uint64_t* rows_empty = rows_full + RS;    // [RS] ... consumed by S^T, dP^T
+    uint64_t* t_full = rows_empty + RS;       // [TS] Q^T, dO^T, row terms of a pair loaded
+    uint64_t* t_empty = t_full + TS;          // [TS] ... consumed by dV, dK
+    uint64_t* kvu_full = t_empty + TS;        // unit's K, V rows loaded
     uint64_t* kvu_empty = kvu_full + 1;       // unit's K, V rows consumed
     uint64_t* s_full = kvu_empty + 1;         // S^T, dP^T in TMEM
     uint64_t* s_free = s_full + 1;            // S^T, dP^T read
@@ -419,18 +467,22 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
     const TcArgs& g = a.geo;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&st_fullb[s], 1);
-            mbar_init(&st_empty[s], 1);
+        for (int s = 0; s < RS; ++s) {
+            mbar_init(&rows_full[s], 1);
+            mbar_init(&rows_empty[s], 1);
+        }
+        for (int s = 0; s < TS; ++s) {
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], 1);
         }
         mbar_init(kvu_full, 1);
         mbar_init(kvu_empty, 1);
         mbar_init(s_full, 1);
-        mbar_init(s_free, 256);
-        mbar_init(pd_full, 256);
+        mbar_init(s_free, bw::kCompute);
+        mbar_init(pd_full, bw::kCompute);
         mbar_init(pd_done, 1);
         mbar_init(unit_done, 1);
-        mbar_init(acc_free, 256);
+        mbar_init(acc_free, bw::kCompute);
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -445,56 +497,69 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
     const uint32_t tmem = *tmem_base_smem;
     const int n_units = *a.n_units;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------------------------ TMA producers
+        // warp 0: each unit's K, V rows, then the Q and dO rows of its pairs;
+        // warp 2: the transposed Q, dO tiles and the row terms of its pairs
+        const bool rows = warp == 0;
+        const int depth = rows ? RS : TS;
+        uint64_t* full = rows ? rows_full : t_full;
+        uint64_t* empty = rows ? rows_empty : t_empty;
         const bool leader = tc::elect_one();
-        uint32_t pc = 0;  // pairs issued by this CTA
+        uint32_t pc = 0;  // pairs issued by this warp
         uint32_t issued_mask = 0, phase_mask = 0;
         int kvu_loads = 0;
         bool ok = true;
         int ui = 0;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++ui) {
             const bw::Unit x = bw::load_unit(a.units, u);
-            if (ui > 0 && !mbar_wait_warp(kvu_empty, (ui - 1) & 1, abort_flag)) { ok = false; break; }
-            if (leader) {
-                int32_t krow;
-                int lo, hi;
-                bw::key_item(g, x, &krow, &lo, &hi);
-                const CUtensorMap* mk = x.kind == 1 ? &g.tm_sk : (x.kind == 2 ? &g.tm_lk : &g.tm_k);
-                const CUtensorMap* mv = x.kind == 1 ? &a.tm_sv : (x.kind == 2 ? &a.tm_lv : &a.tm_v);
-                mbar_arrive_expect_tx(kvu_full, 2 * kT);
-                tma_load_2d(sK, mk, kvu_full, 0, krow);
-                tma_load_2d(sV, mv, kvu_full, 0, krow);
+            if (rows) {
+                if (ui > 0 && !mbar_wait_warp(kvu_empty, (ui - 1) & 1, abort_flag)) { ok = false; break; }
+                if (leader) {
+                    int32_t krow;
+                    int lo, hi;
+                    bw::key_item(g, x, &krow, &lo, &hi);
+                    const CUtensorMap* mk = x.kind == 1 ? &g.tm_sk : (x.kind == 2 ? &g.tm_lk : &g.tm_k);
+                    const CUtensorMap* mv = x.kind == 1 ? &a.tm_sv : (x.kind == 2 ? &a.tm_lv : &a.tm_v);
+                    mbar_arrive_expect_tx(kvu_full, 2 * kT);
+                    tma_load_2d(sK, mk, kvu_full, 0, krow);
+                    tma_load_2d(sV, mv, kvu_full, 0, krow);
+                }
+                ++kvu_loads;
             }
-            ++kvu_loads;
             const int npairs = x.end - x.first;
             for (int n = 0; n < npairs; ++n, ++pc) {
-                const uint32_t s = pc % STAGES, ph = (pc / STAGES) & 1u;
-                if (!mbar_wait_warp(&st_empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+                const uint32_t s = pc % depth, ph = (pc / depth) & 1u;
+                if (!mbar_wait_warp(&empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
                 if (leader) {
                     const int i = bw::unit_query_tile(a, x, n);
-                    int32_t qrow;
-                    int nq;
-                    bw::query_tile(g, x.h, i, &qrow, &nq);
                     const int64_t ti = (int64_t)x.h * g.nt + i;
-                    uint8_t* d = sRing + s * Lay::kStage;
-                    mbar_arrive_expect_tx(&st_fullb[s], 4 * kT + 1024);
-                    tma_load_2d(d, &g.tm_q, &st_fullb[s], 0, qrow);
-                    tma_load_2d(d + kT, &a.tm_do, &st_fullb[s], 0, qrow);
-                    tma_load_2d(d + 2 * kT, &a.tm_qt, &st_fullb[s], 0, (int32_t)(ti * 64));
-                    tma_load_2d(d + 2 * kT + kT / 2, &a.tm_qt, &st_fullb[s], 64, (int32_t)(ti * 64));
-                    tma_load_2d(d + 3 * kT, &a.tm_dot, &st_fullb[s], 0, (int32_t)(ti * 64));
-                    tma_load_2d(d + 3 * kT + kT / 2, &a.tm_dot, &st_fullb[s], 64, (int32_t)(ti * 64));
-                    bulk_load(d + 4 * kT, a.lse2t + ti * 128, 512, &st_fullb[s]);
-                    bulk_load(d + 4 * kT + 512, a.dt + ti * 128, 512, &st_fullb[s]);
+                    if (rows) {
+                        int32_t qrow;
+                        int nq;
+                        bw::query_tile(g, x.h, i, &qrow, &nq);
+                        uint8_t* d = sRows + s * Lay::kRowStage;
+                        mbar_arrive_expect_tx(&full[s], 2 * kT);
+                        tma_load_2d(d, &g.tm_q, &full[s], 0, qrow);
+                        tma_load_2d(d + kT, &a.tm_do, &full[s], 0, qrow);
+                    } else {
+                        uint8_t* d = sTr + s * Lay::kTrStage;
+                        mbar_arrive_expect_tx(&full[s], 2 * kT + 1024);
+                        tma_load_2d(d, &a.tm_qt, &full[s], 0, (int32_t)(ti * 64));
+                        tma_load_2d(d + kT / 2, &a.tm_qt, &full[s], 64, (int32_t)(ti * 64));
+                        tma_load_2d(d + kT, &a.tm_dot, &full[s], 0, (int32_t)(ti * 64));
+                        tma_load_2d(d + kT + kT / 2, &a.tm_dot, &full[s], 64, (int32_t)(ti * 64));
+                        bulk_load(d + 2 * kT, a.lse2t + ti * 128, 512, &full[s]);
+                        bulk_load(d + 2 * kT + 512, a.dt + ti * 128, 512, &full[s]);
+                    }
                 }
                 issued_mask |= 1u << s;
                 phase_mask = (phase_mask & ~(1u << s)) | (ph << s);
             }
         }
         if (!ok) {
-            for (int s = 0; s < STAGES; ++s)
-                if ((issued_mask >> s) & 1u) tc::drain_wait(&st_fullb[s], (phase_mask >> s) & 1u);
+            for (int s = 0; s < depth; ++s)
+                if ((issued_mask >> s) & 1u) tc::drain_wait(&full[s], (phase_mask >> s) & 1u);
             if (kvu_loads > 0) tc::drain_wait(kvu_full, (kvu_loads - 1) & 1);
         }
     } else if (warp == 1) {
@@ -503,8 +568,10 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
         bool ok = true, any_mma = false;
         const uint64_t dkd = smem_desc_sw128(smem_u32(sK), 16, 1024);
         const uint64_t dvd = smem_desc_sw128(smem_u32(sV), 16, 1024);
-        const uint64_t d0 = smem_desc_sw128(smem_u32(sRing), 16, 1024);
-        constexpr uint64_t kStep = (uint64_t)Lay::kStage >> 4;
+        const uint64_t dr0 = smem_desc_sw128(smem_u32(sRows), 16, 1024);
+        const uint64_t dt0 = smem_desc_sw128(smem_u32(sTr), 16, 1024);
+        constexpr uint64_t kRowStep = (uint64_t)Lay::kRowStage >> 4;
+        constexpr uint64_t kTrStep = (uint64_t)Lay::kTrStage >> 4;
         constexpr uint64_t kTile16 = (uint64_t)kT >> 4;
         uint32_t pc = 0;
         int ui = 0;
@@ -514,12 +581,12 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
             if (!mbar_wait_warp(kvu_full, ui & 1, abort_flag)) { ok = false; break; }
             for (int n = 0; n <= npairs && ok; ++n) {
                 if (n < npairs) {
-                    const uint32_t gp = pc + n, s = gp % STAGES, ph = (gp / STAGES) & 1u;
-                    if (!mbar_wait_warp(&st_fullb[s], ph, abort_flag)) { ok = false; break; }
+                    const uint32_t gp = pc + n, s = gp % RS, ph = (gp / RS) & 1u;
+                    if (!mbar_wait_warp(&rows_full[s], ph, abort_flag)) { ok = false; break; }
                     if (gp > 0 && !mbar_wait_warp(s_free, (gp - 1) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     if (leader) {
-                        const uint64_t dst = d0 + s * kStep;
+                        const uint64_t dst = dr0 + s * kRowStep;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)  // S^T = K Q^T
                             umma_ss(tmem + Lay::colS, dkd + 2 * kk, dst + 2 * kk, tc::kIdescS, kk > 0);
@@ -527,6 +594,7 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
                         for (int kk = 0; kk < 4; ++kk)  // dP^T = V dO^T
                             umma_ss(tmem + Lay::colDP, dvd + 2 * kk, dst + kTile16 + 2 * kk, tc::kIdescS, kk > 0);
                         umma_commit(s_full);
+                        umma_commit(&rows_empty[s]);
                         if (n == npairs - 1) umma_commit(kvu_empty);
                     }
                     __syncwarp();
@@ -534,13 +602,14 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
                 }
                 if (n >= 1) {
                     const int m = n - 1;
-                    const uint32_t gp = pc + m, s = gp % STAGES;
+                    const uint32_t gp = pc + m, s = gp % TS, ph = (gp / TS) & 1u;
                     if (!mbar_wait_warp(pd_full, gp & 1, abort_flag)) { ok = false; break; }
                     if (m == 0 && ui > 0 && !mbar_wait_warp(acc_free, (ui - 1) & 1, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait_warp(&t_full[s], ph, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     if (leader) {
-                        const uint64_t dqt = d0 + s * kStep + 2 * kTile16;
-                        const uint64_t ddot = d0 + s * kStep + 3 * kTile16;
+                        const uint64_t dqt = dt0 + s * kTrStep;
+                        const uint64_t ddot = dqt + kTile16;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {  // dV += P^T dO
                             const uint64_t off = (uint64_t)((kk >> 2) * (8192 >> 4) + (kk & 3) * 2);
@@ -553,7 +622,7 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
                             umma_ts(tmem + Lay::colDK, tmem + Lay::colDS + 8 * kk, dqt + off, tc::kIdescPV,
                                     (m > 0 || kk > 0));
                         }
-                        umma_commit(&st_empty[s]);
+                        umma_commit(&t_empty[s]);
                         umma_commit(pd_done);
                         if (m == npairs - 1) umma_commit(unit_done);
                     }
@@ -569,14 +638,15 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------------ P^T, dS^T (thread = key row)
-        const int hc = (warp - 4) >> 2;  // query columns [64 hc, 64 hc + 64)
+        const int hc = (warp - 4) >> 2;  // query columns [32 hc, 32 hc + 32)
         const int quad = warp & 3;
         const int t = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t tS = tmem + Lay::colS + lane_off + hc * 64;
-        const uint32_t tDP = tmem + Lay::colDP + lane_off + hc * 64;
-        const uint32_t tP = tmem + Lay::colP + lane_off + hc * 32;
-        const uint32_t tDS = tmem + Lay::colDS + lane_off + hc * 32;
+        const uint32_t tS = tmem + Lay::colS + lane_off + hc * 32;
+        const uint32_t tDP = tmem + Lay::colDP + lane_off + hc * 32;
+        const uint32_t tP = tmem + Lay::colP + lane_off + hc * 16;
+        const uint32_t tDS = tmem + Lay::colDS + lane_off + hc * 16;
+        const float2 scale2 = make_float2(g.scale_log2, g.scale_log2);
         const int words = g.ntp >> 5;
         uint32_t pc = 0;
         bool ok = true;
@@ -586,8 +656,9 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
             const int npairs = x.end - x.first;
             const int j_lm = x.item * 128 + t;  // landmark chunks: this row's tile
             const float bias = x.kind == 2 ? __ldg(g.lbias2 + j_lm) : 0.0f;
+            const float2 bias2 = make_float2(bias, bias);
             for (int n = 0; n < npairs; ++n) {
-                const uint32_t gp = pc + n, s = gp % STAGES;
+                const uint32_t gp = pc + n, s = gp % TS;
                 bool masked = false;
                 if (x.kind == 2) {
                     const int i = bw::unit_query_tile(a, x, n);
@@ -595,60 +666,59 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
                     masked = (w >> (j_lm & 31)) & 1u;
                 }
                 if (!mbar_wait_warp(s_full, gp & 1, abort_flag)) { ok = false; break; }
-                // the stage's row terms came by bulk copy: observe its barrier directly (already
-                // complete; it cannot be re-armed before this pair's pd_full arrives)
-                if (!mbar_wait_warp(&st_fullb[s], (gp / STAGES) & 1u, abort_flag)) { ok = false; break; }
+                // the pair's row terms come with its transposed tiles (bulk copy): observe that
+                // barrier directly (it cannot be re-armed before this pair's pd_full arrives)
+                if (!mbar_wait_warp(&t_full[s], (gp / TS) & 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const float* lse2s = reinterpret_cast<const float*>(sRing + s * Lay::kStage + 4 * kT);
-                const float* ds_ = lse2s + 128;
-                uint32_t pp[32], pd[32];
+                uint32_t sv[32], dp[32];
+                tmem_ld_32x32b_x32(tS, sv);
+                tmem_ld_32x32b_x32(tDP, dp);
+                tmem_ld_wait(sv);
+                reg_fence(dp);
+                tc_fence_before();
+                mbar_arrive(s_free);  // the next pair's products may overwrite S^T and dP^T now
+                const float2* l2s = reinterpret_cast<const float2*>(sTr + s * Lay::kTrStage + 2 * kT) + hc * 16;
+                const float2* d2s = l2s + 64;
+                uint32_t pp[16], pd[16];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t sv[32], dp[32];
-                    tmem_ld_32x32b_x32(tS + half * 32, sv);
-                    tmem_ld_32x32b_x32(tDP + half * 32, dp);
-                    tmem_ld_wait(sv);
-                    reg_fence(dp);
-                    if (half == 1) {
-                        tc_fence_before();
-                        mbar_arrive(s_free);
+                for (int c2 = 0; c2 < 16; ++c2) {
+                    const float2 l2 = l2s[c2];
+                    const float2 nb = __fadd2_rn(bias2, make_float2(-l2.x, -l2.y));
+                    const float2 xv =
+                        __ffma2_rn(make_float2(__uint_as_float(sv[2 * c2]), __uint_as_float(sv[2 * c2 + 1])), scale2, nb);
+                    float2 p;
+                    if ((c2 & 7) >= 8 - SA_EXP2_FMA_PAIRS_PER8) {
+                        p = exp2_poly2(xv);
+                    } else {
+                        p.x = ex2_approx(xv.x);
+                        p.y = ex2_approx(xv.y);
                     }
-                    const int c0 = hc * 64 + half * 32;
-#pragma unroll
-                    for (int u2 = 0; u2 < 32; u2 += 2) {
-                        float p2[2], d2[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int c = c0 + u2 + e;
-                            const float xv = fmaf(__uint_as_float(sv[u2 + e]), g.scale_log2, bias) - lse2s[c];
-                            const float p = masked ? 0.0f : ex2_approx(xv);
-                            p2[e] = p;
-                            d2[e] = p * (__uint_as_float(dp[u2 + e]) - ds_[c]);
-                        }
-                        pp[half * 16 + u2 / 2] = pack_bf16x2(p2[0], p2[1]);
-                        pd[half * 16 + u2 / 2] = pack_bf16x2(d2[0], d2[1]);
-                    }
+                    if (masked) p = make_float2(0.0f, 0.0f);
+                    const float2 dd = d2s[c2];
+                    const float2 ds = __fmul2_rn(
+                        p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * c2]), __uint_as_float(dp[2 * c2 + 1])),
+                                      make_float2(-dd.x, -dd.y)));
+                    pp[c2] = pack_bf16x2(p.x, p.y);
+                    pd[c2] = pack_bf16x2(ds.x, ds.y);
                 }
                 if (gp > 0) {
                     if (!mbar_wait_warp(pd_done, (gp - 1) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                 }
-                tmem_st_32x32b_x32(tP, pp);
-                tmem_st_32x32b_x32(tDS, pd);
+                tmem_st_32x32b_x16(tP, pp);
+                tmem_st_32x32b_x16(tDS, pd);
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(pd_full);
             }
             if (!ok) break;
-            // ---- epilogue: warpgroup 0 adds the unit's dV rows, warpgroup 1 its dK rows
+            // ---- epilogue: warpgroups 0, 1 add the unit's dV rows (dims 0-31, 32-63), 2, 3 its dK rows
             if (!mbar_wait_warp(unit_done, ui & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            uint32_t acc0[32], acc1[32];
-            const uint32_t tA = tmem + (hc == 0 ? Lay::colDV : Lay::colDK) + lane_off;
-            tmem_ld_32x32b_x32(tA, acc0);
-            tmem_ld_32x32b_x32(tA + 32, acc1);
-            tmem_ld_wait(acc0);
-            reg_fence(acc1);
+            uint32_t acc[32];
+            const uint32_t tA = tmem + (hc < 2 ? Lay::colDV : Lay::colDK) + lane_off + (hc & 1) * 32;
+            tmem_ld_32x32b_x32(tA, acc);
+            tmem_ld_wait(acc);
             tc_fence_before();
             mbar_arrive(acc_free);
             int32_t krow;
@@ -657,30 +727,24 @@ __global__ void __launch_bounds__(384, 1) attn_bwd_dkv_kernel(const __grid_const
             float* dst = nullptr;
             if (t >= lo && t < hi) {
                 if (x.kind == 0) {
-                    dst = (hc == 0 ? a.dv32 : a.dk32) + ((int64_t)krow + t) * 64;
+                    dst = (hc < 2 ? a.dv32 : a.dk32) + ((int64_t)krow + t) * 64;
                 } else if (x.kind == 1) {
                     const int sr = x.item * 128 + t;
                     const int tok = (sr / g.n_sink) * g.tokens + sr % g.n_sink;
-                    dst = (hc == 0 ? a.dv32 : a.dk32) + ((int64_t)x.h * g.L + tok) * 64;
+                    dst = (hc < 2 ? a.dv32 : a.dk32) + ((int64_t)x.h * g.L + tok) * 64;
                 } else {
-                    dst = (hc == 0 ? a.dvbar : a.dkbar) + ((int64_t)x.h * g.ntp + j_lm) * 64;
+                    dst = (hc < 2 ? a.dvbar : a.dkbar) + ((int64_t)x.h * g.ntp + j_lm) * 64;
                 }
             }
             if (dst) {
-                const float mul = hc == 0 ? 1.0f : a.scale;
-                float4* d4 = reinterpret_cast<float4*>(dst);
+                const float mul = hc < 2 ? 1.0f : a.scale;
+                float4* d4 = reinterpret_cast<float4*>(dst) + (hc & 1) * 8;
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4)
-                    atomicAdd(d4 + q4, make_float4(__uint_as_float(acc0[4 * q4 + 0]) * mul,
-                                                   __uint_as_float(acc0[4 * q4 + 1]) * mul,
-                                                   __uint_as_float(acc0[4 * q4 + 2]) * mul,
-                                                   __uint_as_float(acc0[4 * q4 + 3]) * mul));
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4)
-                    atomicAdd(d4 + 8 + q4, make_float4(__uint_as_float(acc1[4 * q4 + 0]) * mul,
-                                                       __uint_as_float(acc1[4 * q4 + 1]) * mul,
-                                                       __uint_as_float(acc1[4 * q4 + 2]) * mul,
-                                                       __uint_as_float(acc1[4 * q4 + 3]) * mul));
+                    atomicAdd(d4 + q4, make_float4(__uint_as_float(acc[4 * q4 + 0]) * mul,
+                                                   __uint_as_float(acc[4 * q4 + 1]) * mul,
+                                                   __uint_as_float(acc[4 * q4 + 2]) * mul,
+                                                   __uint_as_float(acc[4 * q4 + 3]) * mul));
             }
             pc += npairs;
         }
