@@ -40,8 +40,8 @@ struct __align__(64) BwdArgs {
     TcArgs geo;
     CUtensorMap tm_do, tm_v, tm_sv, tm_lv;  // dO rows, V rows, sink V rows, landmark V rows
     CUtensorMap tm_qt, tm_dot;              // transposed query tiles of Q and dO [bh*nt*64][128]
-    const float* lse2t;                     // [bh][nt][128] LSE*log2(e) per query tile row, +inf past the tile
-    const float* dt;                        // [bh][nt][128] rowsum(dO*O), 0 past the tile
+    const float* lse2t;                     // [bh][nt][128] -LSE*log2(e) per query tile row, -inf past the tile
+    const float* dt;                        // [bh][nt][128] -rowsum(dO*O), 0 past the tile
     const uint32_t* listed_bits;            // [bh][nt][ntp/32] bit j: tile j is listed (landmark mode)
     const int4* units;                      // {h, kind << 24 | item, first, end}
     const int32_t* n_units;
@@ -80,8 +80,8 @@ struct QLay {
 struct KVLay {
     static constexpr int RS = 3, TS = 2;
     static constexpr int kK = 0, kV = kT;
-    static constexpr int kRows = 2 * kT, kRowStage = 2 * kT;                  // [RS] Q rows, dO rows
-    static constexpr int kTr = kRows + RS * kRowStage, kTrStage = 2 * kT + 1024;  // [TS] Q^T, dO^T, lse2, D
+    static constexpr int kRows = 2 * kT, kRowStage = 2 * kT + 1024;  // [RS] Q rows, dO rows, -lse2[128], -D[128]
+    static constexpr int kTr = kRows + RS * kRowStage, kTrStage = 2 * kT;  // [TS] Q^T, dO^T
     static constexpr int kBars = kTr + TS * kTrStage;
     static constexpr int kNumBars = 2 * RS + 2 * TS + 9;
     static constexpr int kMisc = kBars + 8 * kNumBars;
@@ -274,15 +274,15 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_consta
         const uint32_t tDP = tmem + Lay::colDP + lane_off + hc * 32;
         const uint32_t tDS = tmem + Lay::colDS + lane_off + hc * 16;
         const uint32_t tDQ = tmem + Lay::colDQ + lane_off + hc * 16;
-        float lse2 = INFINITY, drow = 0.0f;
+        float nlse2 = -INFINITY, ndrow = 0.0f;  // -LSE (base 2) and -D of this row
         if (sl.active) {
             const int64_t ti = ((int64_t)sl.h * g.nt + sl.i) * 128 + r;
-            lse2 = __ldg(a.lse2t + ti);
-            drow = __ldg(a.dt + ti);
+            nlse2 = __ldg(a.lse2t + ti);
+            ndrow = __ldg(a.dt + ti);
         }
         const float2 scale2 = make_float2(g.scale_log2, g.scale_log2);
-        const float2 nl2 = make_float2(-lse2, -lse2);
-        const float2 nd2 = make_float2(-drow, -drow);
+        const float2 nl2 = make_float2(nlse2, nlse2);
+        const float2 nd2 = make_float2(ndrow, ndrow);
         bool ok = true;
         int lm_ptr = 0;
         for (int n = 0; n < n_items; ++n) {
@@ -317,12 +317,8 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_consta
                     const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * u]), __uint_as_float(sv[2 * u + 1])),
                                                 scale2, nl2);
                     float2 p;
-                    if ((u & 7) >= 8 - SA_EXP2_FMA_PAIRS_PER8) {
-                        p = exp2_poly2(x);
-                    } else {
-                        p.x = ex2_approx(x.x);
-                        p.y = ex2_approx(x.y);
-                    }
+                    p.x = ex2_approx(x.x);
+                    p.y = ex2_approx(x.y);
                     const float2 d = __fmul2_rn(
                         p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * u]), __uint_as_float(dp[2 * u + 1])), nd2));
                     pk[u] = pack_bf16x2(d.x, d.y);
@@ -343,9 +339,9 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_consta
                         } else {
                             valid = c >= it.lo && c < it.hi;
                         }
-                        const float x = fmaf(__uint_as_float(sv[2 * u + e]), g.scale_log2, b) - lse2;
+                        const float x = fmaf(__uint_as_float(sv[2 * u + e]), g.scale_log2, b) + nlse2;
                         const float p = valid ? ex2_approx(x) : 0.0f;
-                        d2[e] = p * (__uint_as_float(dp[2 * u + e]) - drow);
+                        d2[e] = p * (__uint_as_float(dp[2 * u + e]) + ndrow);
                     }
                     pk[u] = pack_bf16x2(d2[0], d2[1]);
                 }
@@ -451,9 +447,9 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dkv_kernel(const __grid_const
     uint8_t* sRows = smem + Lay::kRows;
     uint8_t* sTr = smem + Lay::kTr;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBars);
-    uint64_t* rows_full = bars;               // [RS] Q, dO rows of a pair loaded
-    uint64_t* rows_empty = rows_full + RS;    // [RS] ... consumed by S^T, dP^T
-    uint64_t* t_full = rows_empty + RS;       // [TS] Q^T, dO^T, row terms of a pair loaded
+    uint64_t* rows_full = bars;               // [RS] Q, dO rows and row terms of a pair loaded
+    uint64_t* rows_empty = rows_full + RS;    // [RS] ... consumed by S^T, dP^T and the elementwise warps
+    uint64_t* t_full = rows_empty + RS;       // [TS] Q^T, dO^T of a pair loaded
     uint64_t* t_empty = t_full + TS;          // [TS] ... consumed by dV, dK
     uint64_t* kvu_full = t_empty + TS;        // unit's K, V rows loaded
     uint64_t* kvu_empty = kvu_full + 1;       // unit's K, V rows consumed
@@ -469,7 +465,7 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dkv_kernel(const __grid_const
     if (threadIdx.x == 0) {
         for (int s = 0; s < RS; ++s) {
             mbar_init(&rows_full[s], 1);
-            mbar_init(&rows_empty[s], 1);
+            mbar_init(&rows_empty[s], 1 + bw::kCompute);  // the products' commit + every reader of the row terms
         }
         for (int s = 0; s < TS; ++s) {
             mbar_init(&t_full[s], 1);
@@ -499,8 +495,8 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dkv_kernel(const __grid_const
 
     if (warp == 0 || warp == 2) {
         // ------------------------------------------------------------------ TMA producers
-        // warp 0: each unit's K, V rows, then the Q and dO rows of its pairs;
-        // warp 2: the transposed Q, dO tiles and the row terms of its pairs
+        // warp 0: each unit's K, V rows, then the Q and dO rows and row terms of its pairs;
+        // warp 2: the transposed Q, dO tiles of its pairs
         const bool rows = warp == 0;
         const int depth = rows ? RS : TS;
         uint64_t* full = rows ? rows_full : t_full;
@@ -539,18 +535,18 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dkv_kernel(const __grid_const
                         int nq;
                         bw::query_tile(g, x.h, i, &qrow, &nq);
                         uint8_t* d = sRows + s * Lay::kRowStage;
-                        mbar_arrive_expect_tx(&full[s], 2 * kT);
+                        mbar_arrive_expect_tx(&full[s], 2 * kT + 1024);
                         tma_load_2d(d, &g.tm_q, &full[s], 0, qrow);
                         tma_load_2d(d + kT, &a.tm_do, &full[s], 0, qrow);
+                        bulk_load(d + 2 * kT, a.lse2t + ti * 128, 512, &full[s]);
+                        bulk_load(d + 2 * kT + 512, a.dt + ti * 128, 512, &full[s]);
                     } else {
                         uint8_t* d = sTr + s * Lay::kTrStage;
-                        mbar_arrive_expect_tx(&full[s], 2 * kT + 1024);
+                        mbar_arrive_expect_tx(&full[s], 2 * kT);
                         tma_load_2d(d, &a.tm_qt, &full[s], 0, (int32_t)(ti * 64));
                         tma_load_2d(d + kT / 2, &a.tm_qt, &full[s], 64, (int32_t)(ti * 64));
                         tma_load_2d(d + kT, &a.tm_dot, &full[s], 0, (int32_t)(ti * 64));
                         tma_load_2d(d + kT + kT / 2, &a.tm_dot, &full[s], 64, (int32_t)(ti * 64));
-                        bulk_load(d + 2 * kT, a.lse2t + ti * 128, 512, &full[s]);
-                        bulk_load(d + 2 * kT + 512, a.dt + ti * 128, 512, &full[s]);
                     }
                 }
                 issued_mask |= 1u << s;
@@ -658,7 +654,7 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dkv_kernel(const __grid_const
             const float bias = x.kind == 2 ? __ldg(g.lbias2 + j_lm) : 0.0f;
             const float2 bias2 = make_float2(bias, bias);
             for (int n = 0; n < npairs; ++n) {
-                const uint32_t gp = pc + n, s = gp % TS;
+                const uint32_t gp = pc + n, s = gp % RS;
                 bool masked = false;
                 if (x.kind == 2) {
                     const int i = bw::unit_query_tile(a, x, n);
@@ -666,41 +662,47 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dkv_kernel(const __grid_const
                     masked = (w >> (j_lm & 31)) & 1u;
                 }
                 if (!mbar_wait_warp(s_full, gp & 1, abort_flag)) { ok = false; break; }
-                // the pair's row terms come with its transposed tiles (bulk copy): observe that
-                // barrier directly (it cannot be re-armed before this pair's pd_full arrives)
-                if (!mbar_wait_warp(&t_full[s], (gp / TS) & 1u, abort_flag)) { ok = false; break; }
+                // the pair's row terms came with its row tiles (bulk copy): observe that barrier
+                // directly (the stage is not re-armed before this thread's arrival on rows_empty)
+                if (!mbar_wait_warp(&rows_full[s], (gp / RS) & 1u, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t sv[32], dp[32];
-                tmem_ld_32x32b_x32(tS, sv);
-                tmem_ld_32x32b_x32(tDP, dp);
-                tmem_ld_wait(sv);
-                reg_fence(dp);
-                tc_fence_before();
-                mbar_arrive(s_free);  // the next pair's products may overwrite S^T and dP^T now
-                const float2* l2s = reinterpret_cast<const float2*>(sTr + s * Lay::kTrStage + 2 * kT) + hc * 16;
-                const float2* d2s = l2s + 64;
+                // S^T, dP^T in two 16-column halves (fewer live registers): the next pair's S^T
+                // product queues behind this pair's predecessor's dV, dK products in the tensor
+                // pipe anyway, so holding S^T a little longer costs nothing
+                // row terms of this warpgroup's 32 query columns: -LSE (base 2) and -D
+                const float2* nls = reinterpret_cast<const float2*>(sRows + s * Lay::kRowStage + 2 * kT) + hc * 16;
+                const float2* nds = nls + 64;
                 uint32_t pp[16], pd[16];
 #pragma unroll
-                for (int c2 = 0; c2 < 16; ++c2) {
-                    const float2 l2 = l2s[c2];
-                    const float2 nb = __fadd2_rn(bias2, make_float2(-l2.x, -l2.y));
-                    const float2 xv =
-                        __ffma2_rn(make_float2(__uint_as_float(sv[2 * c2]), __uint_as_float(sv[2 * c2 + 1])), scale2, nb);
-                    float2 p;
-                    if ((c2 & 7) >= 8 - SA_EXP2_FMA_PAIRS_PER8) {
-                        p = exp2_poly2(xv);
-                    } else {
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t sv[16], dp[16];
+                    tmem_ld_32x32b_x16(tS + half * 16, sv);
+                    tmem_ld_32x32b_x16(tDP + half * 16, dp);
+                    tmem_ld_wait16(sv);
+                    tmem_ld_wait16(dp);
+                    if (half == 1) {
+                        tc_fence_before();
+                        mbar_arrive(s_free);  // the next pair's products may overwrite S^T and dP^T now
+                    }
+#pragma unroll
+                    for (int c2 = 0; c2 < 8; ++c2) {
+                        const int cc = half * 8 + c2;
+                        const float2 nl = nls[cc];
+                        const float2 nb = x.kind == 2 ? __fadd2_rn(bias2, nl) : nl;
+                        const float2 xv = __ffma2_rn(
+                            make_float2(__uint_as_float(sv[2 * c2]), __uint_as_float(sv[2 * c2 + 1])), scale2, nb);
+                        float2 p;
                         p.x = ex2_approx(xv.x);
                         p.y = ex2_approx(xv.y);
+                        if (masked) p = make_float2(0.0f, 0.0f);
+                        const float2 ds = __fmul2_rn(
+                            p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * c2]), __uint_as_float(dp[2 * c2 + 1])),
+                                          nds[cc]));
+                        pp[cc] = pack_bf16x2(p.x, p.y);
+                        pd[cc] = pack_bf16x2(ds.x, ds.y);
                     }
-                    if (masked) p = make_float2(0.0f, 0.0f);
-                    const float2 dd = d2s[c2];
-                    const float2 ds = __fmul2_rn(
-                        p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * c2]), __uint_as_float(dp[2 * c2 + 1])),
-                                      make_float2(-dd.x, -dd.y)));
-                    pp[c2] = pack_bf16x2(p.x, p.y);
-                    pd[c2] = pack_bf16x2(ds.x, ds.y);
                 }
+                mbar_arrive(&rows_empty[s]);  // row terms read: the stage may be refilled once the products are done
                 if (gp > 0) {
                     if (!mbar_wait_warp(pd_done, (gp - 1) & 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -760,8 +762,9 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dkv_kernel(const __grid_const
 
 // ------------------------------------------------------------------------------ preparation
 
-// Per query tile row: LSE in base-2 units (+inf past the tile or where no key was attended)
-// and D = rowsum(dO * O) (0 past the tile); eight threads per row, 16 bytes each.
+// Per query tile row, negated for the kernels' fused multiply-adds: -LSE in base-2 units (-inf
+// past the tile or where no key was attended) and -D = -rowsum(dO * O) (0 past the tile); eight
+// threads per row, 16 bytes each.
 __global__ void __launch_bounds__(256) bwd_rows_kernel(const __nv_bfloat16* o, const __nv_bfloat16* d_o,
                                                        const float* lse, float* lse2t, float* dt, int32_t bh,
                                                        int32_t nt, int32_t tpf, int32_t tokens, int32_t L) {
@@ -773,7 +776,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const __nv_bfloat16* o, c
     const int h = (int)(hi_ / nt), i = (int)(hi_ % nt);
     const int f = i / tpf, slot = i % tpf;
     const int nq = min(128, tokens - slot * 128);
-    float d = 0.0f, l2 = INFINITY;
+    float d = 0.0f, l2 = -INFINITY;
     if (in_range && r < nq) {
         const int64_t row = (int64_t)h * L + (int64_t)f * tokens + slot * 128 + r;
         const uint4 ov = __ldg(reinterpret_cast<const uint4*>(o + row * 64) + part);
@@ -785,14 +788,14 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const __nv_bfloat16* o, c
             d = fmaf(__uint_as_float(ow[e] & 0xFFFF0000u), __uint_as_float(gw[e] & 0xFFFF0000u), d);
         }
         const float lv = __ldg(lse + row);
-        if (isfinite(lv)) l2 = lv * 1.4426950408889634f;
+        if (isfinite(lv)) l2 = -lv * 1.4426950408889634f;
     }
     d += __shfl_xor_sync(0xffffffffu, d, 1);
     d += __shfl_xor_sync(0xffffffffu, d, 2);
     d += __shfl_xor_sync(0xffffffffu, d, 4);
     if (in_range && part == 0) {
         lse2t[idx] = l2;
-        dt[idx] = r < nq ? d : 0.0f;
+        dt[idx] = r < nq ? -d : 0.0f;
     }
 }
 
