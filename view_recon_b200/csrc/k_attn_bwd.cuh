@@ -289,15 +289,22 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_consta
             const int j_cur = n < sl.cnt ? __ldg(sl.list + n) : 0;
             const tc::Item it = tc::get_item_j(g, sl, n, j_cur);
             if (it.kind < 0 && threadIdx.x == 128) sa_flag_error(SA_ERR_BAD_LIST);
-            uint32_t mw[4] = {0u, 0u, 0u, 0u};  // landmark chunk: listed tiles
+            // validity of this warpgroup's 32 key columns [32 hc, 32 hc + 32): the tile's valid rows,
+            // or for a landmark chunk the tiles the list does not hold
+            uint32_t vmask;
             if (it.kind == 2) {
-                const int c_lo = it.chunk * 128;
+                const int c_lo = it.chunk * 128, w_lo = c_lo + 32 * hc;
+                uint32_t listed = 0u;
                 while (lm_ptr < sl.cnt) {
                     const int j = __ldg(sl.list + lm_ptr);
                     if (j >= c_lo + 128) break;
-                    if (j >= c_lo) mw[(j - c_lo) >> 5] |= 1u << (j & 31);
+                    if (j >= w_lo && j < w_lo + 32) listed |= 1u << (j - w_lo);
                     ++lm_ptr;
                 }
+                vmask = ~listed;
+            } else {
+                const int lo = max(0, it.lo - 32 * hc), hi = min(32, it.hi - 32 * hc);
+                vmask = hi <= lo ? 0u : ((hi - lo == 32 ? 0xFFFFFFFFu : ((1u << (hi - lo)) - 1u)) << lo);
             }
             if (!mbar_wait_warp(sd_full, n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
@@ -309,8 +316,7 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_consta
             tc_fence_before();
             mbar_arrive(sd_free);  // the next item's products may overwrite S and dP now
             uint32_t pk[16];
-            const int c0 = hc * 32;
-            if (it.kind >= 0 && it.kind <= 1 && it.lo == 0 && it.hi == 128) {
+            if (it.kind != 2 && vmask == 0xFFFFFFFFu) {
                 // whole tile attended: no mask, no bias
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
@@ -324,26 +330,20 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_consta
                     pk[u] = pack_bf16x2(d.x, d.y);
                 }
             } else {
-                // partial tile, sink chunk tail, landmark chunk or skipped entry: per-column terms
+                // partial tile, sink chunk tail, landmark chunk (per-column bias) or skipped entry
+                const float2* b2p = it.kind == 2
+                    ? reinterpret_cast<const float2*>(g.lbias2 + it.chunk * 128 + 32 * hc) : nullptr;
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
-                    float d2[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int c = c0 + 2 * u + e;
-                        bool valid;
-                        float b = 0.0f;
-                        if (it.kind == 2) {
-                            valid = ((mw[c >> 5] >> (c & 31)) & 1u) == 0u;
-                            b = __ldg(g.lbias2 + it.chunk * 128 + c);
-                        } else {
-                            valid = c >= it.lo && c < it.hi;
-                        }
-                        const float x = fmaf(__uint_as_float(sv[2 * u + e]), g.scale_log2, b) + nlse2;
-                        const float p = valid ? ex2_approx(x) : 0.0f;
-                        d2[e] = p * (__uint_as_float(dp[2 * u + e]) + ndrow);
-                    }
-                    pk[u] = pack_bf16x2(d2[0], d2[1]);
+                    const float2 nb = b2p ? __fadd2_rn(nl2, __ldg(b2p + u)) : nl2;
+                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[2 * u]), __uint_as_float(sv[2 * u + 1])),
+                                                scale2, nb);
+                    float2 p;
+                    p.x = ((vmask >> (2 * u)) & 1u) ? ex2_approx(x.x) : 0.0f;
+                    p.y = ((vmask >> (2 * u + 1)) & 1u) ? ex2_approx(x.y) : 0.0f;
+                    const float2 d = __fmul2_rn(
+                        p, __fadd2_rn(make_float2(__uint_as_float(dp[2 * u]), __uint_as_float(dp[2 * u + 1])), nd2));
+                    pk[u] = pack_bf16x2(d.x, d.y);
                 }
             }
             if (n > 0) {
