@@ -306,9 +306,9 @@ sa_status sa_sga_fwd(const sa_shape* shape, int32_t grid_h, int32_t grid_w, int3
                      void* o, float* lse_or_null, sa_stream_t stream);
 
 /* Test facility for the failure path (not for production use): while enable != 0, later
- * launches of the tensor-core attention kernel (bf16, tile 128) on the current device never
- * issue the first query-tile load of their first CTA, so that CTA's MMA warp waits for data
- * that cannot arrive.  The wait runs out after the wait limit, the CTA drains what it has in
+ * launches of the tensor-core attention kernels (bf16, tile 128: the forward and the dQ kernel
+ * of sa_sparse_attn_bwd) on the current device never issue the first query-tile load of their
+ * first CTA, so that CTA's MMA warp waits for data that cannot arrive.  The wait runs out after the wait limit, the CTA drains what it has in
  * flight and exits, and sa_check_device_error reports SA_ERR_TIMEOUT; the outputs of such a
  * launch are undefined and the device stays usable.  Returns SA_ERR_CUDA if the setting
  * cannot be written. */

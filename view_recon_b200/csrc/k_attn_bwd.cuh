@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_consta
         const bool leader = tc::elect_one();
         uint32_t issued_mask = 0, phase_mask = 0;
         bool ok = true;
-        if (rows && n_items > 0 && leader) {
+        const bool withhold = g_sa_test_withhold != 0 && blockIdx.x == 0;  // failure-path test facility
+        if (rows && n_items > 0 && leader && !withhold) {
             mbar_arrive_expect_tx(q_full, 2 * kT);
             tma_load_2d(sQ, &g.tm_q, q_full, 0, sl.qrow);
             tma_load_2d(sDO, &a.tm_do, q_full, 0, sl.qrow);
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(640, 1) attn_bwd_dq_kernel(const __grid_consta
         if (!ok) {
             for (int s = 0; s < depth; ++s)
                 if ((issued_mask >> s) & 1u) tc::drain_wait(&full[s], (phase_mask >> s) & 1u);
-            if (rows && n_items > 0) tc::drain_wait(q_full, 0);
+            if (rows && n_items > 0 && !withhold) tc::drain_wait(q_full, 0);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
