@@ -96,3 +96,55 @@ def test_backward_vggt16_full_call_two_heads():
     w = VGGT_S16
     layer, data, do_h, got = run_case(w, seed=11)
     compare(w, layer, data, do_h, got, [0, w.heads - 1])
+
+
+def _rows_of(t, h, rows):
+    import torch
+    return H.from_device(t[h, torch.as_tensor(np.asarray(rows), device=t.device)])
+
+
+@pytest.mark.parametrize("wname", ["vggt_s128_n1374", "vggt_s512_n1374_landmark"])
+def test_backward_large_workload_sampled(wname):
+    """The benchmark's layer call at 128 frames (k = 130) and 512 frames (landmarks), forward and
+    backward over all 16 heads; compared on samples the oracle can finish in seconds: dq of
+    seeded query tiles of the first and last head (first and last frame, a frame's sink tile and
+    partial tile among them), and at 128 frames dk, dv of one key tile per head, whose rows the
+    oracle completes by running every query tile that lists it.  (A key tile's landmark gradient at
+    512 frames gathers from nearly every query tile, beyond a sampled check.)"""
+    import torch
+    from synth.workloads import BY_NAME
+    from view_recon_b200 import sa
+    w = BY_NAME[wname]
+    data = H.inputs(w)
+    layer, (q, k, v) = H.run_gpu(w, data)
+    do_h = bf16_normal((w.heads, w.L, 64), 13)
+    d_o = H.to_device(do_h, "bf16")
+    dq, dk, dv = layer.backward(q, k, v, d_o)
+    torch.cuda.synchronize()
+    assert sa.sa_check_device_error() == 0
+    g = H.geometry(w)
+    tpf, nt = w.tpf, g.nt
+    rng = np.random.default_rng(21)
+    tiles = sorted(set([0, tpf - 1, nt - tpf, nt - 1, (w.frames // 2) * tpf + 3] +
+                       rng.choice(nt, size=3, replace=False).tolist()))
+    for h in (0, w.heads - 1):
+        Qh, Kh, Vh = (orc.to_f64(data[x][h:h + 1]) for x in ("q", "k", "v"))
+        dOh = orc.to_f64(do_h[h:h + 1])
+        idx = H.from_device(layer.buf.kept_idx[h]).astype(np.int64)
+        cnt = H.from_device(layer.buf.kept_cnt[h]).astype(np.int64)
+        kept = [idx[i, :cnt[i]] for i in range(nt)]
+        ref_q, _, _ = orc.attend_backward(g, Qh, Kh, Vh, [kept], dOh, 0.125, w.landmark,
+                                          items=[(0, i) for i in tiles])
+        rows = np.concatenate([g.tile_rows(i) for i in tiles])
+        check_grad("dq h=%d" % h, _rows_of(dq, h, rows), ref_q[0, rows])
+        if w.landmark:
+            continue
+        # one key tile per head: an interior tile of a random frame, then a frame's sink-holding tile
+        j_pick = int(rng.integers(1, tpf)) + tpf * int(rng.integers(0, w.frames)) if h == 0 else 2 * tpf
+        for j in (j_pick,):
+            users = [i for i in range(nt) if j in set(kept[i].tolist())]
+            _, ref_k, ref_v = orc.attend_backward(g, Qh, Kh, Vh, [kept], dOh, 0.125, False,
+                                                  items=[(0, i) for i in users])
+            kr = g.tile_key_rows(j)  # non-sink rows: complete with these query tiles
+            check_grad("dk h=%d j=%d" % (h, j), _rows_of(dk, h, kr), ref_k[0, kr])
+            check_grad("dv h=%d j=%d" % (h, j), _rows_of(dv, h, kr), ref_v[0, kr])
