@@ -25,6 +25,10 @@
 //                        and adds the unit's dK, dV rows to fp32 accumulators (float4 atomics;
 //                        a key item split over several units, and every sink row, receives
 //                        several contributions).
+// Warp roles of both kernels (640 threads, one CTA per SM): warp 0 and warp 2 the TMA producers
+// of the two operand rings, warp 1 the tcgen05.mma issuer (it also owns the TMEM allocation),
+// warp 3 idle, warpgroups 1-4 the elementwise work (32 of the 128 columns each; a thread owns one
+// row of the 128-row tile).
 // Every operand is staged K-major in shared memory by TMA (128-byte swizzle); the transposed
 // tiles (Q^T, dO^T, K^T) are written once per call by the transpose kernel of the forward.
 // Every wait is bounded (g_sa_wait_limit_ns) and drains what the role has in flight.
@@ -61,9 +65,10 @@ constexpr int kThreads = 640;   // warps 0-3 control, warpgroups 1-4 the element
 constexpr int kCompute = 512;
 
 // Operands come through two rings per kernel, each with its own producer warp: the row tiles
-// read by the S / dP products (released as soon as those complete) and the transposed tiles
-// read by the gradient products (released after them), so that the next tiles' copies start
-// early and their latency stays off the tensor pipe's path.
+// read by the S / dP products (released as soon as those complete; in the dK/dV kernel also
+// once every elementwise thread has read the per-row terms that ride with them) and the
+// transposed tiles read by the gradient products (released after them), so that the next
+// tiles' copies start early and their latency stays off the tensor pipe's path.
 struct QLay {
     static constexpr int RS = 4, TS = 3;
     static constexpr int kQ = 0, kDO = kT;
