@@ -500,3 +500,25 @@ def test_backward_landmarks_exact_when_tile_rows_are_identical():
     _, dk, _ = orc.attend_backward(g, q, k, v, kept, do, 0.6, landmark=True)
     _, dk_d, _ = orc.dense_backward(q, k, v, do, 0.6)
     np.testing.assert_allclose(dk, dk_d, rtol=0, atol=1e-12)
+
+
+def test_backward_restricted_items_complete_what_they_cover():
+    """Running only some query tiles gives the full backward's dq on those tiles, and the full
+    dk, dv on a key tile's non-sink rows when every query tile that lists it is included (the
+    sampled comparisons at large sizes rely on both)."""
+    g, q, k, v = _tiny_case(80, frames=4, tokens=9, tile=4, n_sink=1, bh=1, d=3)
+    qb, kb, _, _, _, _ = orc.pool(g, q, k, v)
+    kept = orc.select(g, orc.scores(qb, kb), 2)
+    do = rnd(q.shape, 81)
+    dq, dk, dv = orc.attend_backward(g, q, k, v, kept, do, 0.5)
+    tiles = [0, 5, g.nt - 1]
+    dq_s, _, _ = orc.attend_backward(g, q, k, v, kept, do, 0.5, items=[(0, i) for i in tiles])
+    rows = np.concatenate([g.tile_rows(i) for i in tiles])
+    np.testing.assert_allclose(dq_s[0, rows], dq[0, rows], rtol=0, atol=1e-14)
+    for j in (1, 6):
+        users = [i for i in range(g.nt) if j in set(kept[0][i].tolist())]
+        assert 0 < len(users) < g.nt
+        _, dk_s, dv_s = orc.attend_backward(g, q, k, v, kept, do, 0.5, items=[(0, i) for i in users])
+        kr = g.tile_key_rows(j)
+        np.testing.assert_allclose(dk_s[0, kr], dk[0, kr], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(dv_s[0, kr], dv[0, kr], rtol=0, atol=1e-14)
