@@ -148,3 +148,24 @@ def test_backward_large_workload_sampled(wname):
             kr = g.tile_key_rows(j)  # non-sink rows: complete with these query tiles
             check_grad("dk h=%d j=%d" % (h, j), _rows_of(dk, h, kr), ref_k[0, kr])
             check_grad("dv h=%d j=%d" % (h, j), _rows_of(dv, h, kr), ref_v[0, kr])
+
+
+@pytest.mark.parametrize("landmark", [False, True])
+def test_backward_per_head_budgets(landmark):
+    """Per-head budgets (k = 0, 3, 9): rows of the smaller budgets hold fewer tiles than max_kept,
+    the rest of each row being -1; every gradient of every head against the oracle."""
+    import torch
+    from view_recon_b200 import sa
+    from view_recon_b200.pipeline import SparseGlobalAttention
+    w = Workload("per_head", 5, 300, 3, 64, 128, 5, "bf16", 9, landmark, False, 256, 0, 0.7)
+    data = H.inputs(w)
+    q, k, v = (H.to_device(data[x], "bf16") for x in ("q", "k", "v"))
+    layer = SparseGlobalAttention(w.heads, w.frames, w.tokens, [0, 3, 9], landmark=landmark)
+    layer.forward(q, k, v)
+    do_h = bf16_normal((w.heads, w.L, 64), 17)
+    dq, dk, dv = layer.backward(q, k, v, H.to_device(do_h, "bf16"))
+    torch.cuda.synchronize()
+    assert sa.sa_check_device_error() == 0
+    cnt = H.from_device(layer.buf.kept_cnt)
+    assert cnt[0].max() < layer.max_kept == cnt[2].max()  # short rows are present
+    compare(w, layer, data, do_h, (H.from_device(dq), H.from_device(dk), H.from_device(dv)), range(w.heads))
