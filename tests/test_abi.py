@@ -159,3 +159,33 @@ def test_backward_host_checks(lib):
     shp = sa.shape(16, 16, 1374, 64, 128, 5, "bf16")
     assert sa.sa_sparse_attn_bwd_workspace_size(shp, 46, True) > sa.sa_sparse_attn_bwd_workspace_size(shp, 46, False)
     assert sa.sa_sparse_attn_bwd_workspace_size(shp, 100, False) > sa.sa_sparse_attn_bwd_workspace_size(shp, 46, False)
+
+
+def test_backward_workspace_layout():
+    """The backward's workspace is the documented sum of its parts (each rounded to 256 bytes)."""
+    from view_recon_b200 import sa
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    bh, S, N, max_kept = 16, 16, 1374, 46
+    nt, L = S * 11, S * N
+    M = bh * nt
+    tile = 64 * 128 * 2
+    sink_tiles = -(-S * 5 // 128)
+    chunks_q = -(-nt // 32)
+
+    def expect(landmark):
+        ntp = -(-nt // 128) * 128
+        lm_chunks = ntp // 128 if landmark else 0
+        units_cap = bh * (sink_tiles + lm_chunks) * chunks_q + (M * max_kept) // 32 + M + 1
+        parts = [M * 128 * 4, M * 128 * 4, M * tile, M * tile, M * tile, bh * sink_tiles * tile,
+                 bh * ntp * 128 if landmark else 0, bh * ntp * 128 if landmark else 0,
+                 bh * lm_chunks * tile, bh * lm_chunks * tile, ntp * 4 if landmark else 0,
+                 M * (ntp // 32) * 4 if landmark else 0, M * 4, M * 4, M * max_kept * 4, units_cap * 16, 16,
+                 bh * L * 64 * 4, bh * L * 64 * 4,
+                 bh * ntp * 64 * 4 if landmark else 0, bh * ntp * 64 * 4 if landmark else 0]
+        return sum(a256(p) for p in parts)
+
+    shp = sa.shape(bh, S, N, 64, 128, 5, "bf16")
+    assert sa.sa_sparse_attn_bwd_workspace_size(shp, max_kept, False) == expect(False)
+    assert sa.sa_sparse_attn_bwd_workspace_size(shp, max_kept, True) == expect(True)
+    assert sa.sa_sparse_attn_bwd_workspace_size(shp, 0, False) == 0          # max_kept out of range
+    assert sa.sa_sparse_attn_bwd_workspace_size(shp, nt + 1, False) == 0
