@@ -178,7 +178,10 @@ sa_status sa_select_topk_per_head(const sa_shape* shape, const float* scores_or_
  *   Limit: nt <= 32768 (the scratch holds at least 64 whole score rows); larger shapes
  *          return SA_ERR_UNSUPPORTED.
  *   Set-up: the first call on a device looks up the scratch array's device address (a host-
- *          side runtime query); make that first call before any stream capture begins.
+ *          side runtime query); make that first call before any stream capture begins.  The
+ *          address is kept for the life of the process: after cudaDeviceReset the module may
+ *          load at another address, so this call is not valid across a device reset (nor is
+ *          any other entry point, whose one-time kernel attributes a reset also clears).
  *   Sharing: all calls on a device use the same array and it keeps the last call's contents
  *          (every score row is written before it is read, so nothing needs clearing).  Calls
  *          whose kernels overlap on the GPU (e.g. on different streams) race on it.

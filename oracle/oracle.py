@@ -160,10 +160,11 @@ def scores(q_bar: np.ndarray, k_bar: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------- step 3: selection
 
 def candidates(g: Geometry, i: int) -> np.ndarray:
-    """Key tiles that query tile i may choose: outside its own frame, with a non-sink row."""
-    forced = g.own_frame_tiles(i)
-    cand = np.setdiff1d(np.arange(g.nt), forced)
-    return np.array([j for j in cand if g.key_count(int(j)) > 0], dtype=np.int64)
+    """Key tiles that query tile i may choose: outside its own frame, with a non-sink row.
+    (Which rows of a tile are sinks depends only on the tile's slot within its frame.)"""
+    slot_has_key = np.array([g.key_count(slot) > 0 for slot in range(g.tpf)], dtype=bool)
+    j = np.arange(g.nt, dtype=np.int64)
+    return j[(j // g.tpf != g.frame_of_tile(i)) & slot_has_key[j % g.tpf]]
 
 
 def select_row(g: Geometry, s_row: np.ndarray, i: int, k: int) -> np.ndarray:

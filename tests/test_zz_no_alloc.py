@@ -65,6 +65,9 @@ def test_noalloc_selection_equals_workspace_selection_twice():
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
+    """The scratch holds 64 rows of the longest row any selection accepts (32768 tiles; a
+    static assertion in the library keeps it so), so that row limit is the binding one: a
+    longer row is refused before any launch."""
     import torch
     from view_recon_b200 import sa
     lib = sa.load()

@@ -826,9 +826,12 @@ __global__ void bwd_scan_lists_kernel(const int32_t* kept_idx, const int32_t* ke
 // One block: CSR offsets of the reverse lists (per key tile, over all heads), the unit table
 // (fixed sink / landmark units first, then each key tile's list in runs of kBwdChunk) and the
 // number of units.  fill[] starts at each list's offset for bwd_fill_lists_kernel.
+// Writes at most units_cap units: a plan that would need more (possible only for malformed lists)
+// is cut at the capacity, reported as SA_ERR_BAD_LIST, and the unit count clamped to it.
 __global__ void __launch_bounds__(1024) bwd_plan_kernel(const int32_t* rev_cnt, int32_t* fill, int4* units,
                                                         int32_t* n_units, int32_t bh, int32_t nt,
-                                                        int32_t n_sink_tiles, int32_t n_lm_chunks) {
+                                                        int32_t n_sink_tiles, int32_t n_lm_chunks,
+                                                        int64_t units_cap) {
     __shared__ int64_t s_e[1024], s_u[1024];
     const int64_t M = (int64_t)bh * nt;
     const int64_t per = (M + 1023) / 1024;
@@ -857,11 +860,16 @@ __global__ void __launch_bounds__(1024) bwd_plan_kernel(const int32_t* rev_cnt, 
         const int c = rev_cnt[x];
         fill[x] = (int32_t)e0;
         const int h = (int)(x / nt), j = (int)(x % nt);
-        for (int q = 0; q * kBwdChunk < c; ++q)
+        for (int q = 0; q * kBwdChunk < c; ++q) {
+            if (u0 >= units_cap) {
+                sa_flag_error(SA_ERR_BAD_LIST);
+                break;
+            }
             units[u0++] = make_int4(h, j, (int32_t)(e0 + q * kBwdChunk), (int32_t)(e0 + min(c, (q + 1) * kBwdChunk)));
+        }
         e0 += c;
     }
-    for (int64_t f = threadIdx.x; f < n_fixed; f += 1024) {
+    for (int64_t f = threadIdx.x; f < n_fixed && f < units_cap; f += 1024) {
         const int64_t per_head = (n_sink_tiles + n_lm_chunks) * chunks_q;
         const int h = (int)(f / per_head);
         const int64_t r = f % per_head;
@@ -870,7 +878,7 @@ __global__ void __launch_bounds__(1024) bwd_plan_kernel(const int32_t* rev_cnt, 
         const int item = it < n_sink_tiles ? it : it - n_sink_tiles;
         units[f] = make_int4(h, (kind << 24) | item, q * kBwdChunk, min(nt, (q + 1) * kBwdChunk));
     }
-    if (threadIdx.x == 1023) *n_units = (int32_t)(n_fixed + s_u[1023]);
+    if (threadIdx.x == 1023) *n_units = (int32_t)min(units_cap, n_fixed + s_u[1023]);
 }
 
 __global__ void bwd_fill_lists_kernel(const int32_t* kept_idx, const int32_t* kept_cnt, int32_t max_kept,

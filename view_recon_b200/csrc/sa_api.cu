@@ -16,6 +16,9 @@
 
 // Fixed scratch of sa_select_topk_noalloc: one block of score rows (2 Mi floats = 8 MiB).
 constexpr long long kNoallocScratchFloats = 1ll << 21;
+// 64 rows of the longest row any selection accepts (SEL_MAX_NT) fit, so SEL_MAX_NT is the
+// binding limit of the no-allocation call.
+static_assert(kNoallocScratchFloats >= 64ll * SEL_MAX_NT, "scratch must hold 64 rows of SEL_MAX_NT scores");
 static __device__ __align__(256) float g_sa_noalloc_scores[kNoallocScratchFloats];
 
 namespace {
@@ -1044,7 +1047,8 @@ sa_status sa_sparse_attn_bwd(const sa_shape* shape, const void* q, const void* k
         if ((st = launch_status()) != SA_OK) return st;
         bwd_plan_kernel<<<1, 1024, 0, stream>>>(rev_cnt, fill, reinterpret_cast<int4*>(base + w.units),
                                                 reinterpret_cast<int32_t*>(base + w.n_units), (int32_t)g.bh,
-                                                (int32_t)g.nt, (int32_t)w.n_sink_tiles, (int32_t)w.n_lm_chunks);
+                                                (int32_t)g.nt, (int32_t)w.n_sink_tiles, (int32_t)w.n_lm_chunks,
+                                                (int64_t)w.units_cap);
         if ((st = launch_status()) != SA_OK) return st;
         bwd_fill_lists_kernel<<<blocks, 256, 0, stream>>>(kept_idx, kept_cnt, max_kept, (int32_t)g.bh, (int32_t)g.nt,
                                                           fill, reinterpret_cast<int32_t*>(base + w.rev));
