@@ -198,6 +198,60 @@ def select_per_head(g: Geometry, s: np.ndarray, k_per_head):
     return [[select_row(g, s[h, i], i, int(k_per_head[h])) for i in range(g.nt)] for h in range(s.shape[0])]
 
 
+# ----------------------------------------------------------------------------- per-head budgets
+
+def candidate_entropy(g: Geometry, s_row: np.ndarray, i: int, scale: float) -> float:
+    """Entropy (natural log) of the softmax of scale * s_row over the candidate tiles of query
+    tile i: H = -sum_j p_j ln p_j with p_j = exp(x_j) / sum_c exp(x_c), x = scale * s.
+    Written as ln Z - sum_j p_j (x_j - m) with m = max x and Z = sum_j exp(x_j - m), which is
+    the same quantity without a logarithm of a vanishing p.  No candidate: 0."""
+    cand = candidates(g, i)
+    if len(cand) == 0:
+        return 0.0
+    x = scale * s_row[cand]
+    m = x.max()
+    w = np.exp(x - m)
+    z = w.sum()
+    return float(np.log(z) - (w / z * (x - m)).sum())
+
+
+def head_budgets(g: Geometry, q_bar: np.ndarray, k_bar: np.ndarray, scale: float, beta: float,
+                 k_lo: int, k_hi: int):
+    """Per-head budgets from an online statistic of the head's own pooled scores.
+
+    Heads differ in how concentrated their attention is, and the budget of each head is
+    adapted online ("SAF3R" abstract: per-head sparsity from offline profiling and online
+    adaptation).  The statistic of head h is the mean perplexity of its query tiles,
+        P_h = (1/nt) sum_i exp(H_i),
+    H_i the entropy of the softmax of scale * s_ij over the candidate tiles j of tile i (0 for
+    a tile without candidates, so that it adds nothing): the effective number of candidates the
+    tile-level attention spreads over.  The budget keeps that many tiles, scaled by beta:
+        k_h = min(k_hi, max(k_lo, floor(beta * P_h + 1/2))).
+    Uniform scores give P_h = the candidate count (every candidate kept when beta >= 1); one
+    dominant candidate per row gives P_h -> 1.  Returns (P [bh], k [bh] int64)."""
+    s = scores(q_bar, k_bar)
+    bh = s.shape[0]
+    perp = np.zeros((bh,))
+    for h in range(bh):
+        tot = 0.0
+        for i in range(g.nt):
+            tot += np.exp(candidate_entropy(g, s[h, i], i, scale)) if len(candidates(g, i)) else 0.0
+        perp[h] = tot / g.nt
+    k = np.minimum(k_hi, np.maximum(k_lo, np.floor(beta * perp + 0.5))).astype(np.int64)
+    return perp, k
+
+
+def budget_matches(perp_ref: float, beta: float, k_lo: int, k_hi: int, got: int, rel: float = 1e-4) -> bool:
+    """A GPU budget computed in f32 is accepted iff it equals the fp64 rule's, or beta * P lies
+    within rel (relative) of a rounding boundary n + 1/2 and the GPU took the other side."""
+    want = int(min(k_hi, max(k_lo, np.floor(beta * perp_ref + 0.5))))
+    if got == want:
+        return True
+    x = beta * perp_ref
+    frac_dist = abs((x - 0.5) - np.round(x - 0.5))
+    return abs(got - want) == 1 and frac_dist <= rel * max(1.0, abs(x))
+
+
 def max_kept(g: Geometry, k: int) -> int:
     """Length of every kept list: own-frame tiles plus min(k, candidates)."""
     n_cand = (g.frames - 1) * sum(1 for slot in range(g.tpf) if g.key_count(slot) > 0)

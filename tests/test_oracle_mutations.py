@@ -35,6 +35,10 @@ PIN_TESTS = [
     lambda: pins.test_backward_all_tiles_is_dense(2),
     lambda: pins.test_backward_landmarks_exact_when_tile_rows_are_identical(),
     lambda: pins.test_backward_matches_finite_differences(True, 1, 1),
+    lambda: pins.test_candidate_entropy_two_candidates_closed_form(),
+    lambda: pins.test_candidate_entropy_bruteforce_excludes_own_frame_and_keyless_tiles(),
+    lambda: pins.test_head_budgets_uniform_scores_give_the_candidate_count(),
+    lambda: pins.test_head_budgets_mean_of_perplexities_bruteforce(),
 ]
 
 
@@ -232,7 +236,38 @@ def _backward_variant(drop_rowsum=False, share_whole=False, dk_unscaled=False, d
     return attend_backward
 
 
+_candidate_entropy = orc.candidate_entropy
+
+
+def entropy_over_every_tile(g, s_row, i, scale):
+    x = scale * s_row  # slip: own frame and keyless tiles enter the softmax
+    m = x.max()
+    w = np.exp(x - m)
+    z = w.sum()
+    return float(np.log(z) - (w / z * (x - m)).sum())
+
+
+def entropy_unscaled(g, s_row, i, scale):
+    return _candidate_entropy(g, s_row, i, 1.0)  # slip: temperature dropped
+
+
+def entropy_base2(g, s_row, i, scale):
+    return _candidate_entropy(g, s_row, i, scale) / math.log(2.0)  # slip: bits instead of nats
+
+
+def head_budgets_exp_of_mean_entropy(g, q_bar, k_bar, scale, beta, k_lo, k_hi):
+    s = orc.scores(q_bar, k_bar)
+    perp = np.array([math.exp(np.mean([orc.candidate_entropy(g, s[h, i], i, scale) for i in range(g.nt)]))
+                     for h in range(s.shape[0])])  # slip: exp of the mean entropy
+    k = np.minimum(k_hi, np.maximum(k_lo, np.floor(beta * perp + 0.5))).astype(np.int64)
+    return perp, k
+
+
 MUTANTS = {
+    "entropy_over_every_tile": ("candidate_entropy", entropy_over_every_tile),
+    "entropy_unscaled": ("candidate_entropy", entropy_unscaled),
+    "entropy_base2": ("candidate_entropy", entropy_base2),
+    "budget_exp_of_mean_entropy": ("head_budgets", head_budgets_exp_of_mean_entropy),
     "bwd_rowsum_term_dropped": ("attend_backward", _backward_variant(drop_rowsum=True)),
     "bwd_landmark_gradient_not_shared": ("attend_backward", _backward_variant(share_whole=True)),
     "bwd_dk_unscaled": ("attend_backward", _backward_variant(dk_unscaled=True)),

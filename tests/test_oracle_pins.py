@@ -522,3 +522,87 @@ def test_backward_restricted_items_complete_what_they_cover():
         kr = g.tile_key_rows(j)
         np.testing.assert_allclose(dk_s[0, kr], dk[0, kr], rtol=0, atol=1e-14)
         np.testing.assert_allclose(dv_s[0, kr], dv[0, kr], rtol=0, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- per-head budgets
+
+def _entropy_by_hand(probs):
+    return -sum(p * math.log(p) for p in probs if p > 0.0)
+
+
+def test_candidate_entropy_two_candidates_closed_form():
+    """Three frames of one tile each: every query tile has exactly two candidates, whose softmax
+    entropy is written out with math.exp / math.log."""
+    g = orc.Geometry(frames=3, tokens=4, tile=4, n_sink=0)  # tpf 1, nt 3
+    s = np.array([0.3, -1.2, 2.5])
+    for i, tau in ((0, 0.7), (1, 2.0), (2, 0.1)):
+        x = [tau * s[j] for j in range(3) if j != i]
+        z = math.exp(x[0]) + math.exp(x[1])
+        want = _entropy_by_hand([math.exp(x[0]) / z, math.exp(x[1]) / z])
+        assert abs(orc.candidate_entropy(g, s, i, tau) - want) < 1e-12
+
+
+def test_candidate_entropy_bruteforce_excludes_own_frame_and_keyless_tiles():
+    g = orc.Geometry(frames=4, tokens=7, tile=3, n_sink=3)  # slot 0 of every frame is all sinks
+    rng = np.random.default_rng(21)
+    for i in range(g.nt):
+        s = rng.standard_normal(g.nt) * 3
+        cand = [j for j in range(g.nt) if j // g.tpf != i // g.tpf and (j % g.tpf) != 0]
+        z = sum(math.exp(0.5 * s[j]) for j in cand)
+        want = _entropy_by_hand([math.exp(0.5 * s[j]) / z for j in cand])
+        assert abs(orc.candidate_entropy(g, s, i, 0.5) - want) < 1e-12
+
+
+def test_head_budgets_uniform_scores_give_the_candidate_count():
+    """Identical key means make every score of a row equal: the softmax is uniform, its
+    perplexity is the number of candidates, and beta = 1 keeps all of them (the dense budget)."""
+    g = orc.Geometry(frames=5, tokens=300, tile=128, n_sink=5)  # 3 slots, all holding keys
+    rng = np.random.default_rng(3)
+    qb = rng.standard_normal((2, g.nt, 8))
+    kb = np.repeat(rng.standard_normal((2, 1, 8)), g.nt, axis=1)
+    n_cand = (g.frames - 1) * g.tpf
+    perp, k = orc.head_budgets(g, qb, kb, 0.9, 1.0, 0, 10_000)
+    assert np.allclose(perp, n_cand, rtol=0, atol=1e-9)
+    assert k.tolist() == [n_cand, n_cand]
+    _, k = orc.head_budgets(g, qb, kb, 0.9, 0.5, 0, 10_000)
+    assert k.tolist() == [n_cand // 2] * 2                 # floor(beta * P + 1/2), P = 12
+    _, k = orc.head_budgets(g, qb, kb, 0.9, 1.0, 0, 7)
+    assert k.tolist() == [7, 7]                            # clamped above
+    _, k = orc.head_budgets(g, qb, kb, 0.9, 0.01, 5, 100)
+    assert k.tolist() == [5, 5]                            # clamped below
+
+
+def test_head_budgets_one_dominant_candidate():
+    """One candidate far above the rest in every row: perplexity 1, whatever the head."""
+    g = orc.Geometry(frames=3, tokens=8, tile=4, n_sink=0)  # tpf 2, nt 6, 4 candidates per row
+    qb = np.zeros((1, g.nt, 2))
+    qb[0, :, 0] = 1.0
+    kb = np.zeros((1, g.nt, 2))
+    kb[0, [0, 2, 4], 0] = [200.0, 150.0, 100.0]  # each row's best candidate beats the next by >= 50
+    perp, k = orc.head_budgets(g, qb, kb, 1.0, 3.0, 0, 99)
+    assert abs(perp[0] - 1.0) < 1e-12
+    assert k[0] == 3
+
+
+def test_head_budgets_mean_of_perplexities_bruteforce():
+    g = orc.Geometry(frames=3, tokens=5, tile=2, n_sink=1)  # tpf 3, slot 0 holds 1 key row
+    rng = np.random.default_rng(8)
+    qb, kb = rng.standard_normal((3, g.nt, 4)), rng.standard_normal((3, g.nt, 4))
+    perp, k = orc.head_budgets(g, qb, kb, 0.8, 0.7, 1, 6)
+    for h in range(3):
+        tot = 0.0
+        for i in range(g.nt):
+            cand = [j for j in range(g.nt) if j // 3 != i // 3]
+            x = [0.8 * sum(qb[h, i, e] * kb[h, j, e] for e in range(4)) for j in cand]
+            z = sum(math.exp(v) for v in x)
+            tot += math.exp(_entropy_by_hand([math.exp(v) / z for v in x]))
+        assert abs(perp[h] - tot / g.nt) < 1e-10
+        assert k[h] == min(6, max(1, math.floor(0.7 * tot / g.nt + 0.5)))
+
+
+def test_budget_rule_accepts_rounding_boundary_only():
+    assert orc.budget_matches(10.2, 1.0, 0, 99, 10)
+    assert not orc.budget_matches(10.2, 1.0, 0, 99, 11)
+    assert orc.budget_matches(10.5 * (1 + 2e-5), 1.0, 0, 99, 10)   # f32 may round 10.50002 down
+    assert orc.budget_matches(10.5 * (1 - 2e-5), 1.0, 0, 99, 11)
+    assert not orc.budget_matches(10.5 * (1 + 2e-3), 1.0, 0, 99, 10)
