@@ -167,6 +167,33 @@ sa_status sa_select_topk_per_head(const sa_shape* shape, const float* scores_or_
                                   int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept,
                                   void* workspace_or_null, size_t workspace_bytes, sa_stream_t stream);
 
+/* Bytes of workspace sa_head_budgets needs: one f32 per (head, query tile). */
+size_t sa_head_budget_workspace_size(const sa_shape* shape);
+
+/*
+ * Per-head budgets from an online statistic of each head's own pooled scores (SAF3R
+ * abstract: sparsity differs across heads and each head's budget is adapted online).  The
+ * pages give no formula; this call computes, for every head h,
+ *   H_i  = entropy (natural log) of softmax_j(temperature * s_ij) over the candidate tiles j
+ *          of query tile i (the tiles sa_select_topk may choose), 0 without candidates
+ *   P_h  = (1/nt) sum_i exp(H_i)   (mean perplexity: how many candidates a tile spreads over;
+ *          a tile without candidates adds 0)
+ *   k_h  = min(k_hi, max(k_lo, floor(beta * P_h + 1/2)))
+ * with s_ij = q_pool[h][i] . k_pool[h][j] (the f32 FMA chain of sa_tile_scores, recomputed:
+ * no score matrix is read or written).  Outputs, DEVICE memory:
+ *   k_per_head          int32 [bh], 4-byte aligned - ready for sa_select_topk_per_head with
+ *                       k_max = k_hi in the same stream
+ *   perplexity_or_null  f32 [bh] P_h (may be NULL)
+ * temperature > 0 and beta >= 0 finite, 0 <= k_lo <= k_hi, else SA_ERR_INVALID_ARG;
+ * workspace >= sa_head_budget_workspace_size(shape) bytes, 16-byte aligned, else
+ * SA_ERR_WORKSPACE.  Deterministic (fixed summation orders).  Uniform scores give P_h = the
+ * candidate count, so beta = 1 with k_hi at or above it makes that head dense.
+ */
+sa_status sa_head_budgets(const sa_shape* shape, const float* q_pool, const float* k_pool, float temperature,
+                          float beta, int32_t k_lo, int32_t k_hi, int32_t* k_per_head,
+                          float* perplexity_or_null, void* workspace, size_t workspace_bytes,
+                          sa_stream_t stream);
+
 /*
  * sa_select_topk in streamed mode without any caller-provided memory.  No passage of the
  * pages corresponds to this call; it exists for callers that cannot allocate device memory

@@ -189,3 +189,27 @@ def test_backward_workspace_layout():
     assert sa.sa_sparse_attn_bwd_workspace_size(shp, max_kept, True) == expect(True)
     assert sa.sa_sparse_attn_bwd_workspace_size(shp, 0, False) == 0          # max_kept out of range
     assert sa.sa_sparse_attn_bwd_workspace_size(shp, nt + 1, False) == 0
+
+
+def test_head_budget_validation_happens_before_any_launch(lib):
+    from view_recon_b200 import sa
+    shp = sa.shape(2, 4, 300, 64, 128, 5, "bf16")
+    s = ctypes.byref(shp)
+    P = ctypes.c_void_p
+    fake, odd2 = P(0x10000), P(0x10002)
+    nt = sa.sa_num_tiles(shp)
+    assert sa.sa_head_budget_workspace_size(shp) == 2 * nt * 4
+    ws = 2 * nt * 4
+    f = ctypes.c_float
+    ok_args = (f(16.0), f(1.0), 0, 10, fake, None, fake, ws, None)
+    assert lib.sa_head_budgets(s, None, fake, *ok_args) == sa.SA_ERR_INVALID_ARG           # no q_pool
+    assert lib.sa_head_budgets(s, fake, fake, f(16.0), f(1.0), 0, 10, odd2, None, fake, ws,
+                               None) == sa.SA_ERR_INVALID_ARG                            # misaligned budgets
+    assert lib.sa_head_budgets(s, fake, fake, f(0.0), f(1.0), 0, 10, fake, None, fake, ws,
+                               None) == sa.SA_ERR_INVALID_ARG                            # temperature 0
+    assert lib.sa_head_budgets(s, fake, fake, f(16.0), f(-1.0), 0, 10, fake, None, fake, ws,
+                               None) == sa.SA_ERR_INVALID_ARG                            # negative beta
+    assert lib.sa_head_budgets(s, fake, fake, f(16.0), f(1.0), 5, 4, fake, None, fake, ws,
+                               None) == sa.SA_ERR_INVALID_ARG                            # k_lo > k_hi
+    assert lib.sa_head_budgets(s, fake, fake, f(16.0), f(1.0), 0, 10, fake, None, fake, ws - 4,
+                               None) == sa.SA_ERR_WORKSPACE                              # short workspace

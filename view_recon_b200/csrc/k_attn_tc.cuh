@@ -108,12 +108,13 @@ __device__ __forceinline__ Slot make_slot(const TcArgs& a, int item) {
 
 __device__ __forceinline__ Item get_item_j(const TcArgs& a, const Slot& s, int n, int j);
 
+// Item n of slot s, reading its list entry from global memory.
 __device__ __forceinline__ Item get_item(const TcArgs& a, const Slot& s, int n) {
     const int j = (!a.dense && n < s.cnt) ? __ldg(s.list + n) : 0;
     return get_item_j(a, s, n, j);
 }
 
-// Same as get_item with the list entry s.list[n] (when n < s.cnt) supplied by the caller.
+// Item n of slot s; j is the list entry s.list[n] when n < s.cnt (see ListWindow).
 __device__ __forceinline__ Item get_item_j(const TcArgs& a, const Slot& s, int n, int j) {
     Item it;
     it.chunk = 0;
@@ -161,6 +162,28 @@ __device__ __forceinline__ Item get_item_j(const TcArgs& a, const Slot& s, int n
     it.chunk = n;
     return it;
 }
+
+// The slot's kept list, read 32 entries at a time: lane l holds entry 32w + l of the current
+// window w and of the next one (loaded a whole window ahead, so no item waits for a global
+// load); entry n is one warp shuffle.  All 32 lanes must call entry() for every n in order.
+struct ListWindow {
+    int32_t cur, next;
+    __device__ __forceinline__ ListWindow(const TcArgs& a, const Slot& s, int lane) {
+        const bool listed = !a.dense && s.cnt > 0;
+        cur = (listed && lane < s.cnt) ? __ldg(s.list + lane) : 0;
+        next = (listed && 32 + lane < s.cnt) ? __ldg(s.list + 32 + lane) : 0;
+    }
+    __device__ __forceinline__ int entry(const TcArgs& a, const Slot& s, int n, int lane) {
+        if (a.dense || n >= s.cnt) return 0;  // uniform over the warp
+        const int j = __shfl_sync(0xffffffffu, cur, n & 31);
+        if ((n & 31) == 31) {
+            cur = next;
+            const int e = n + 33 + lane;
+            next = e < s.cnt ? __ldg(s.list + e) : 0;
+        }
+        return j;
+    }
+};
 
 // Bounded wait that ignores the abort flag (used only to drain in-flight work).  Copies and
 // MMAs already issued complete in microseconds; the limit is at least 1 s whatever the
@@ -282,14 +305,16 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                 mbar_arrive_expect_tx(q_full, tc::kTileBytes);
                 tma_load_2d(sQ, &a.tm_q, q_full, 0, sl.qrow);
             }
+            tc::ListWindow win(a, sl, lane);
             for (int n = 0; n < n_items; ++n) {
                 const uint32_t s = n % STAGES, ph = (n / STAGES) & 1u;
                 if (!mbar_wait_warp(&kv_empty[s], ph ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
+                const int j_cur = win.entry(a, sl, n, lane);
                 if (leader) {
-                    const tc::Item it = tc::get_item(a, sl, n);
+                    const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
                     const CUtensorMap* mk = it.kind == 1 ? &a.tm_sk : (it.kind == 2 ? &a.tm_lk : &a.tm_k);
                     const CUtensorMap* mv = it.kind == 1 ? &a.tm_svt : (it.kind == 2 ? &a.tm_lvt : &a.tm_vt);
                     uint8_t* dk = sKV + s * 2 * tc::kTileBytes;
@@ -373,9 +398,9 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         int lm_ptr = 0;                                              // landmark chunks: list cursor
+        tc::ListWindow win(a, sl, lane);
         for (int n = 0; n < sl.n_items; ++n) {
-            const int j_cur = (!a.dense && n < sl.cnt) ? __ldg(sl.list + n) : 0;  // (a prefetch one item ahead
-            // measured slower: it lengthens register live ranges in this loop)
+            const int j_cur = win.entry(a, sl, n, lane);
             const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
             if (it.kind < 0 && st == 0) sa_flag_error(SA_ERR_BAD_LIST);  // skipped list entry
             if (!mbar_wait_warp(s_full, n & 1, abort_flag)) { ok = false; break; }
@@ -422,9 +447,17 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                 }
                 mul = 1.0f;
             } else if (it.lo > 0 || it.hi < 128) {
+                // valid columns [lo, hi) as four 32-bit words; one bit test and select per column
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c < it.lo || c >= it.hi) sv[c] = __float_as_uint(-INFINITY);
+                for (int w4 = 0; w4 < 4; ++w4) {
+                    const int b0 = min(max(it.lo - 32 * w4, 0), 32), b1 = min(max(it.hi - 32 * w4, 0), 32);
+                    const uint32_t below_hi = b1 == 32 ? 0xFFFFFFFFu : ((1u << b1) - 1u);
+                    const uint32_t below_lo = b0 == 32 ? 0xFFFFFFFFu : ((1u << b0) - 1u);
+                    const uint32_t valid = below_hi & ~below_lo;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                        if (!((valid >> u) & 1u)) sv[32 * w4 + u] = __float_as_uint(-INFINITY);
+                }
             }
             float mx8[8];
 #pragma unroll

@@ -9,6 +9,7 @@
 #include "k_attn_prep.cuh"
 #include "k_attn_simt.cuh"
 #include "k_attn_tc.cuh"
+#include "k_budget.cuh"
 #include "k_pool.cuh"
 #include "k_scores.cuh"
 #include "k_select.cuh"
@@ -111,6 +112,8 @@ sa_status ensure_attributes() {
                                (int)bw::KVLay::smem_bytes()) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tile_scores_big_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SCORES_BIG_SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(head_stat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BUDGET_SMEM) ==
+          cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SEL_SMEM_BUDGET) == cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -686,6 +689,48 @@ sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, con
         }
     }
     return SA_OK;
+}
+
+size_t sa_head_budget_workspace_size(const sa_shape* shape) {
+    Geo g;
+    if (geo_of(shape, &g) != SA_OK) return 0;
+    return (size_t)g.bh * (size_t)g.nt * 4;
+}
+
+sa_status sa_head_budgets(const sa_shape* shape, const float* q_pool, const float* k_pool, float temperature,
+                          float beta, int32_t k_lo, int32_t k_hi, int32_t* k_per_head, float* perplexity_or_null,
+                          void* workspace, size_t workspace_bytes, sa_stream_t stream) {
+    Geo g;
+    sa_status st = geo_of(shape, &g);
+    if (st != SA_OK) return st;
+    if (!q_pool || !k_pool || !aligned16(q_pool) || !aligned16(k_pool)) return SA_ERR_INVALID_ARG;
+    if (!k_per_head || (reinterpret_cast<uintptr_t>(k_per_head) & 3u)) return SA_ERR_INVALID_ARG;
+    if (perplexity_or_null && (reinterpret_cast<uintptr_t>(perplexity_or_null) & 3u)) return SA_ERR_INVALID_ARG;
+    if (!(temperature > 0.0f) || isinf(temperature) || !(beta >= 0.0f) || isinf(beta)) return SA_ERR_INVALID_ARG;
+    if (k_lo < 0 || k_hi < k_lo) return SA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < sa_head_budget_workspace_size(shape) || !aligned16(workspace))
+        return SA_ERR_WORKSPACE;
+    if (g.bh > 65535 || (g.nt + 127) / 128 > 2147483647ll) return SA_ERR_UNSUPPORTED;
+    if ((st = ensure_attributes()) != SA_OK) return st;
+    BudgetArgs a;
+    a.q_pool = q_pool;
+    a.k_pool = k_pool;
+    a.row_perp = static_cast<float*>(workspace);
+    a.k_per_head = k_per_head;
+    a.perp_out = perplexity_or_null;
+    a.nt = (int32_t)g.nt;
+    a.tpf = (int32_t)g.tpf;
+    a.tile = (int32_t)g.T;
+    a.tokens = (int32_t)g.N;
+    a.n_sink = (int32_t)g.n_sink;
+    a.temperature = temperature;
+    a.beta = beta;
+    a.k_lo = k_lo;
+    a.k_hi = k_hi;
+    head_stat_kernel<<<dim3((unsigned)((g.nt + 127) / 128), (unsigned)g.bh), 256, BUDGET_SMEM, stream>>>(a);
+    if ((st = launch_status()) != SA_OK) return st;
+    head_budget_kernel<<<(unsigned)g.bh, 256, 0, stream>>>(a);
+    return launch_status();
 }
 
 size_t sa_sparse_attn_workspace_size(const sa_shape* shape, int32_t landmark) {

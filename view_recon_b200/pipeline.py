@@ -48,15 +48,25 @@ class SparseGlobalAttention:
     k          key tiles chosen per query tile beyond its own frame's tiles: one budget for every
                head, or a sequence of bh per-head budgets (a budget at or above the candidate
                count makes that head dense)
+    adaptive   None, or a dict(temperature=, beta=, k_lo=) that sets every head's budget on the
+               device from the spread of its own pooled scores (sa_head_budgets) before each
+               selection; k is then the largest budget (k_hi); temperature defaults to tile/sqrt(d)
     landmark   fold every unselected tile into one mean-K/mean-V token (+ln count bias)
     streamed   select without materialising the [bh][nt][nt] score matrix
     """
 
     def __init__(self, bh: int, frames: int, tokens: int, k: int, tile: int = 128, n_sink: int = 5,
                  dtype: str = "bf16", landmark: bool = False, streamed: bool = False, head_dim: int = 64,
-                 device=None, with_lse: bool = True):
+                 device=None, with_lse: bool = True, adaptive=None):
         import torch
         self.shape = sa.shape(bh, frames, tokens, head_dim, tile, n_sink, dtype)
+        self.adaptive = None
+        if adaptive is not None:
+            if not (isinstance(k, int) or getattr(k, "ndim", None) == 0):
+                raise ValueError("with adaptive budgets k is the single largest budget")
+            ad = dict(adaptive)
+            self.adaptive = (float(ad.get("temperature", tile / head_dim ** 0.5)), float(ad.get("beta", 1.0)),
+                             int(ad.get("k_lo", 0)), int(k))
         if isinstance(k, (int,)) or getattr(k, "ndim", None) == 0:
             self.k, self.k_per_head = int(k), None
         else:
@@ -82,6 +92,13 @@ class SparseGlobalAttention:
         attn_bytes = sa.sa_sparse_attn_workspace_size(self.shape, self.landmark)
         self.k_head = (torch.tensor(self.k_per_head, dtype=torch.int32, device=dev)
                        if self.k_per_head is not None else None)
+        self.perplexity = None
+        self.budget_ws = None
+        if self.adaptive is not None:
+            self.k_head = torch.zeros((bh,), dtype=torch.int32, device=dev)
+            self.perplexity = torch.zeros((bh,), dtype=torch.float32, device=dev)
+            self.budget_ws = torch.empty((sa.sa_head_budget_workspace_size(self.shape),), dtype=torch.uint8,
+                                         device=dev)
         self.buf = Buffers(
             q_pool=torch.empty((bh, nt, head_dim), dtype=f32, device=dev),
             k_pool=torch.empty((bh, nt, head_dim), dtype=f32, device=dev),
@@ -108,8 +125,16 @@ class SparseGlobalAttention:
         if not self.streamed:
             sa.sa_tile_scores(self.shape, self.buf.q_pool, self.buf.k_pool, self.buf.scores, stream)
 
+    def budgets(self, stream=None):
+        """Adaptive mode: every head's budget from its own pooled scores (one C call)."""
+        if self.adaptive is not None:
+            tau, beta, k_lo, k_hi = self.adaptive
+            sa.sa_head_budgets(self.shape, self.buf.q_pool, self.buf.k_pool, tau, beta, k_lo, k_hi, self.k_head,
+                               self.perplexity, self.budget_ws, stream)
+
     def select(self, stream=None):
         b = self.buf
+        self.budgets(stream)
         if self.k_head is None:
             sa.sa_select_topk(self.shape, b.scores, b.q_pool, b.k_pool, self.k, b.kept_idx, b.kept_cnt,
                               self.max_kept, b.sel_ws, stream)
@@ -173,6 +198,8 @@ class SparseGlobalAttention:
             n += 2 * self.bh * (-(-self.nt // rows))  # score block + select block
         else:
             n += 2  # scores + select
+        if self.adaptive is not None:
+            n += 2  # per-head statistic + budgets
         n += 1  # attention
         if sa.sa_sparse_attn_workspace_size(self.shape, self.landmark) > 0:
             n += 1  # transposed V tiles

@@ -28,7 +28,8 @@ SA_BF16 = 1
 # every symbol include/sa.h declares
 EXPORTS = [
     "sa_num_tiles", "sa_max_kept", "sa_tile_pool", "sa_tile_scores", "sa_select_workspace_size",
-    "sa_select_topk", "sa_select_topk_per_head", "sa_select_topk_noalloc", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
+    "sa_select_topk", "sa_select_topk_per_head", "sa_select_topk_noalloc", "sa_head_budget_workspace_size",
+    "sa_head_budgets", "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd", "sa_dense_attn_workspace_size",
     "sa_dense_attn_fwd", "sa_sga_workspace_size", "sa_sga_fwd", "sa_sparse_attn_bwd_workspace_size",
     "sa_sparse_attn_bwd",
     "sa_status_string", "sa_check_device_error", "sa_set_wait_limit_ns", "sa_test_withhold_query_load",
@@ -77,6 +78,8 @@ def load(path: str | None = None):
         "sa_select_topk": (i32, [shp, vp, vp, vp, i32, vp, vp, i32, vp, sz, vp]),
         "sa_select_topk_per_head": (i32, [shp, vp, vp, vp, vp, i32, vp, vp, i32, vp, sz, vp]),
         "sa_select_topk_noalloc": (i32, [shp, vp, vp, i32, vp, vp, i32, vp]),
+        "sa_head_budget_workspace_size": (sz, [shp]),
+        "sa_head_budgets": (i32, [shp, vp, vp, ctypes.c_float, ctypes.c_float, i32, i32, vp, vp, vp, sz, vp]),
         "sa_sparse_attn_workspace_size": (sz, [shp, i32]),
         "sa_sparse_attn_fwd": (i32, [shp, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp, vp,
                                      vp]),
@@ -176,6 +179,20 @@ def sa_select_topk_per_head(shp, scores, q_pool, k_pool, k_per_head, k_max, kept
                                         _ptr(k_per_head), int(k_max), _ptr(kept_idx), _ptr(kept_cnt),
                                         int(max_kept), _ptr(workspace), ws_bytes, _stream(stream))
     _check("sa_select_topk_per_head", st)
+
+
+def sa_head_budget_workspace_size(shp) -> int:
+    return int(load().sa_head_budget_workspace_size(ctypes.byref(shp)))
+
+
+def sa_head_budgets(shp, q_pool, k_pool, temperature, beta, k_lo, k_hi, k_per_head, perplexity=None,
+                    workspace=None, stream=None):
+    """k_per_head: int32 device tensor [bh] (written); perplexity: f32 device tensor [bh] or None."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load().sa_head_budgets(ctypes.byref(shp), _ptr(q_pool), _ptr(k_pool), float(temperature), float(beta),
+                                int(k_lo), int(k_hi), _ptr(k_per_head), _ptr(perplexity), _ptr(workspace), ws_bytes,
+                                _stream(stream))
+    _check("sa_head_budgets", st)
 
 
 def sa_select_topk_noalloc(shp, q_pool, k_pool, k, kept_idx, kept_cnt, max_kept, stream=None):
