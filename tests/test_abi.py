@@ -93,7 +93,12 @@ def test_workspace_sizes(lib):
     shp = sa.shape(16, 1024, 1374, 64, 128, 5, "bf16")
     assert sa.sa_select_workspace_size(shp, False) == 0
     ws = sa.sa_select_workspace_size(shp, True)
-    assert 0 < ws <= 64 << 20 and ws % (11264 * 4) == 0  # whole score rows, L2-sized
+    # two buffers of R whole score rows (R a multiple of 128, L2-sized together) + control words
+    R = (24 << 20) // (11264 * 4) // 128 * 128
+    nblk = -(-11264 // R)
+    bufs = 2 * R * 11264 * 4
+    assert R == 512 and ws == bufs + -(-(2 + 2 * 16 * nblk) * 4 // 256) * 256
+    assert ws <= 64 << 20
     shp4 = sa.shape(16, 512, 1374, 64, 128, 5, "bf16")
     vt = 16 * 5632 * 64 * 128 * 2                 # transposed V tiles of every key tile
     sinks = 16 * 20 * 64 * 128 * 2                # 512 frames x 5 sinks = 2560 rows = 20 tiles

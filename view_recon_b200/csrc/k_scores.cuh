@@ -70,24 +70,22 @@ __global__ void __launch_bounds__(256) tile_scores_kernel(ScoreArgs a) {
 
 #define SCORES_BIG_SMEM (2 * 64 * 128 * 4)
 
-// 128 x 128 block per 256-thread CTA; dynamic shared memory SCORES_BIG_SMEM (qT, kT: [64][128]).
-__global__ void __launch_bounds__(256) tile_scores_big_kernel(ScoreArgs a) {
-    extern __shared__ __align__(16) float big_smem[];
-    float* qT = big_smem;             // [64 e][128 rows]
-    float* kT = big_smem + 64 * 128;  // [64 e][128 cols]
+// One 128 x 128 block of scores by the whole 256-thread CTA: rows qb[0 .. rows_valid) and
+// columns kb[0 .. cols_valid) (each a [64] f32 mean), written to ob[r * ldo + c]; smem holds
+// SCORES_BIG_SMEM bytes (qT, kT: [64][128]).  Starts and ends with the CTA converged; the
+// caller synchronises before reusing smem.
+__device__ __forceinline__ void score_block_128(const float* qb, int rows_valid, const float* kb, int cols_valid,
+                                                float* ob, int64_t ldo, float* smem) {
+    float* qT = smem;             // [64 e][128 rows]
+    float* kT = smem + 64 * 128;  // [64 e][128 cols]
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const int h = a.h0 + blockIdx.z;
-    const int r_blk = blockIdx.y * 128;
-    const int c_blk = blockIdx.x * 128;
-    const float* qb = a.q_pool + ((int64_t)h * a.nt + a.i0) * 64;
-    const float* kb = a.k_pool + (int64_t)h * a.nt * 64;
     // consecutive lanes take consecutive rows, so the transposed shared-memory writes of a warp
     // fall into 32 different banks
     for (int idx = threadIdx.x; idx < 128 * 16; idx += 256) {
         const int r = idx & 127, c4 = idx >> 7;  // row r, elements 4 c4 .. 4 c4 + 3
         float4 x = make_float4(0, 0, 0, 0), y = x;
-        if (r_blk + r < a.rows) x = __ldg(reinterpret_cast<const float4*>(qb + (int64_t)(r_blk + r) * 64) + c4);
-        if (c_blk + r < a.nt) y = __ldg(reinterpret_cast<const float4*>(kb + (int64_t)(c_blk + r) * 64) + c4);
+        if (r < rows_valid) x = __ldg(reinterpret_cast<const float4*>(qb + (int64_t)r * 64) + c4);
+        if (r < cols_valid) y = __ldg(reinterpret_cast<const float4*>(kb + (int64_t)r * 64) + c4);
         qT[(4 * c4 + 0) * 128 + r] = x.x;
         qT[(4 * c4 + 1) * 128 + r] = x.y;
         qT[(4 * c4 + 2) * 128 + r] = x.z;
@@ -117,23 +115,34 @@ __global__ void __launch_bounds__(256) tile_scores_big_kernel(ScoreArgs a) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) acc[u][p] = __ffma2_rn(make_float2(qv[u], qv[u]), kv[p], acc[u][p]);
     }
-    float* ob = a.out + (int64_t)blockIdx.z * a.rows * a.ldo;
-    const int c0 = c_blk + tx * 8;
-    const bool vec = ((a.ldo & 3) == 0) && (c0 + 8 <= a.nt);
+    const int c0 = tx * 8;
+    const bool vec = ((ldo & 3) == 0) && (c0 + 8 <= cols_valid) && ((reinterpret_cast<uintptr_t>(ob) & 15u) == 0);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-        const int r = r_blk + ty * 8 + u;
-        if (r >= a.rows) continue;
-        float* dst = ob + (int64_t)r * a.ldo + c0;
+        const int r = ty * 8 + u;
+        if (r >= rows_valid) continue;
+        float* dst = ob + (int64_t)r * ldo + c0;
         if (vec) {
             reinterpret_cast<float4*>(dst)[0] = make_float4(acc[u][0].x, acc[u][0].y, acc[u][1].x, acc[u][1].y);
             reinterpret_cast<float4*>(dst)[1] = make_float4(acc[u][2].x, acc[u][2].y, acc[u][3].x, acc[u][3].y);
         } else {
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-                if (c0 + 2 * p < a.nt) dst[2 * p] = acc[u][p].x;
-                if (c0 + 2 * p + 1 < a.nt) dst[2 * p + 1] = acc[u][p].y;
+                if (c0 + 2 * p < cols_valid) dst[2 * p] = acc[u][p].x;
+                if (c0 + 2 * p + 1 < cols_valid) dst[2 * p + 1] = acc[u][p].y;
             }
         }
     }
+}
+
+// 128 x 128 block per 256-thread CTA; dynamic shared memory SCORES_BIG_SMEM (qT, kT: [64][128]).
+__global__ void __launch_bounds__(256) tile_scores_big_kernel(ScoreArgs a) {
+    extern __shared__ __align__(16) float big_smem[];
+    const int h = a.h0 + blockIdx.z;
+    const int r_blk = blockIdx.y * 128;
+    const int c_blk = blockIdx.x * 128;
+    const float* qb = a.q_pool + ((int64_t)h * a.nt + a.i0 + r_blk) * 64;
+    const float* kb = a.k_pool + ((int64_t)h * a.nt + c_blk) * 64;
+    float* ob = a.out + ((int64_t)blockIdx.z * a.rows + r_blk) * a.ldo + c_blk;
+    score_block_128(qb, a.rows - r_blk, kb, a.nt - c_blk, ob, a.ldo, big_smem);
 }

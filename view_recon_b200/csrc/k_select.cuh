@@ -364,8 +364,13 @@ __device__ __forceinline__ uint32_t sel_find_bin(const uint32_t* hist, uint32_t 
     return total;
 }
 
-__global__ void __launch_bounds__(SEL_BLOCK_THREADS) select_topk_block_kernel(SelectArgs a) {
-    extern __shared__ __align__(16) uint32_t sel_smem[];
+// Selection of one row (head h, query tile i) by the whole 256-thread CTA; sel_smem holds
+// select_block_smem_bytes(nt) bytes.  The row is staged by one bulk copy (cg_rows == false) or,
+// for rows that other CTAs of the same launch have just written, by L2-coherent loads.
+// Returns false when a wait ran out (reported in the error word); the CTA is converged on
+// return either way.
+__device__ __forceinline__ bool select_row_block(const SelectArgs& a, int h, int i, const float* row,
+                                                 bool cg_rows, uint32_t* sel_smem) {
     const int nt = a.nt;
     const int nwords = (nt + 31) >> 5;
     uint32_t* stage = sel_smem;
@@ -381,17 +386,15 @@ __global__ void __launch_bounds__(SEL_BLOCK_THREADS) select_topk_block_kernel(Se
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int h = a.h0 + blockIdx.y, i = a.i0 + blockIdx.x;
-    const float* row = a.scores + ((int64_t)blockIdx.y * a.rows + blockIdx.x) * a.lds;
     const int f0 = (i / a.tpf) * a.tpf, f1 = f0 + a.tpf;  // own-frame tiles [f0, f1)
     const int s0 = a.n_sink / a.tile;                      // slots below s0 hold no key row
 
     // ---- stage the row: one bulk copy for its 16-byte-aligned middle, plain loads for the
     // (at most 3 + 3) scores at either end.  keys[c] = stage[mis + c], so that the copy's
     // destination keys + ha is 16-byte aligned like its source row + ha.
-    const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(row) >> 2) & 3u;
-    const int ha = min(nt, (int)((4u - mis) & 3u));
-    const int n4 = (nt - ha) >> 2;
+    const uint32_t mis = cg_rows ? 0u : (uint32_t)(reinterpret_cast<uintptr_t>(row) >> 2) & 3u;
+    const int ha = cg_rows ? 0 : min(nt, (int)((4u - mis) & 3u));
+    const int n4 = cg_rows ? 0 : (nt - ha) >> 2;
     const int hb = ha + 4 * n4;
     uint32_t* keys = stage + mis;
     if (tid == 0) {
@@ -405,15 +408,19 @@ __global__ void __launch_bounds__(SEL_BLOCK_THREADS) select_topk_block_kernel(Se
             bulk_load(keys + ha, row + ha, (uint32_t)n4 * 16u, &bar);
         }
     }
-    if (tid < ha) keys[tid] = __float_as_uint(__ldg(row + tid));
-    if (tid >= 32 && tid - 32 < nt - hb) keys[hb + tid - 32] = __float_as_uint(__ldg(row + hb + tid - 32));
+    if (cg_rows) {
+        for (int c = tid; c < nt; c += SEL_BLOCK_THREADS) keys[c] = __float_as_uint(__ldcg(row + c));
+    } else {
+        if (tid < ha) keys[tid] = __float_as_uint(__ldg(row + tid));
+        if (tid >= 32 && tid - 32 < nt - hb) keys[hb + tid - 32] = __float_as_uint(__ldg(row + hb + tid - 32));
+    }
 #pragma unroll
     for (int u = 0; u < SEL_BLOCK_H1 / SEL_BLOCK_THREADS; ++u) hist1[u * SEL_BLOCK_THREADS + tid] = 0u;
     for (int w = tid; w < nwords; w += SEL_BLOCK_THREADS) eqmask[w] = 0u;
     __syncthreads();
     if (n4 > 0) {
         const bool ok = mbar_wait(&bar, 0, &abort_flag);
-        if (__syncthreads_or(!ok)) return;  // timed out: the error word says so
+        if (__syncthreads_or(!ok)) return false;  // timed out: the error word says so
     }
 
     // ---- 1. keys in place + first-level histogram (sink slots taken out afterwards)
@@ -553,4 +560,13 @@ __global__ void __launch_bounds__(SEL_BLOCK_THREADS) select_topk_block_kernel(Se
     }
     for (int p = tot + tid; p < a.max_kept; p += SEL_BLOCK_THREADS) out[p] = -1;
     if (tid == 0) a.kept_cnt[(int64_t)h * nt + i] = (int32_t)tot;
+    __syncthreads();  // the CTA's shared memory may be reused right after
+    return true;
+}
+
+__global__ void __launch_bounds__(SEL_BLOCK_THREADS) select_topk_block_kernel(SelectArgs a) {
+    extern __shared__ __align__(16) uint32_t sel_smem[];
+    const int h = a.h0 + blockIdx.y, i = a.i0 + blockIdx.x;
+    const float* row = a.scores + ((int64_t)blockIdx.y * a.rows + blockIdx.x) * a.lds;
+    select_row_block(a, h, i, row, false, sel_smem);
 }

@@ -13,6 +13,7 @@
 #include "k_pool.cuh"
 #include "k_scores.cuh"
 #include "k_select.cuh"
+#include "k_select_stream.cuh"
 #include "k_sga.cuh"
 
 // Fixed scratch of sa_select_topk_noalloc: one block of score rows (2 Mi floats = 8 MiB).
@@ -118,6 +119,9 @@ sa_status ensure_attributes() {
                                SEL_SMEM_BUDGET) == cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)select_block_smem_bytes(SEL_MAX_NT)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(select_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)std::max<size_t>(SCORES_BIG_SMEM, select_block_smem_bytes(SEL_MAX_NT))) ==
+          cudaSuccess;
     // The tensor-core kernel moves registers between its warpgroups (setmaxnreg); that is only
     // satisfiable if the block is launched with at least the registers the split hands out.
     cudaFuncAttributes fa;
@@ -236,11 +240,31 @@ AttnWs attn_ws(const Geo& g, bool dense, bool landmark, int64_t Lk = -1) {
 
 bool use_tc(const Geo& g) { return g.bf16 && g.T == 128 && g.d == 64; }
 
-size_t select_rows_per_block(const Geo& g) {
-    // one block of score rows stays in L2 (about 48 MB), at least 64 rows
-    int64_t r = (48ll << 20) / (g.nt * 4);
-    r = std::max<int64_t>(64, r / 64 * 64);
-    return (size_t)std::min<int64_t>(r, g.nt);
+// Streamed selection: two buffers of R score rows that together stay in L2 (about 48 MB), R a
+// multiple of 128 (whole score tiles), at least 128, at most the row count; then the control
+// words (item counter, abort word, two completion counts per block).
+struct StreamWs {
+    int64_t R, nblk, G, col_tiles, items_per_head;
+    size_t buf, ctl, ctl_bytes, total;
+};
+StreamWs stream_ws(const Geo& g) {
+    StreamWs w;
+    int64_t r = (24ll << 20) / (g.nt * 4);
+    r = std::max<int64_t>(128, r / 128 * 128);
+    w.R = std::min<int64_t>(r, g.nt);
+    w.nblk = (g.nt + w.R - 1) / w.R;
+    w.G = g.bh * w.nblk;
+    w.col_tiles = (g.nt + 127) / 128;
+    w.items_per_head = 0;
+    for (int64_t b = 0; b < w.nblk; ++b) {
+        const int64_t rows = std::min<int64_t>(w.R, g.nt - b * w.R);
+        w.items_per_head += ((rows + 127) / 128) * w.col_tiles + rows;
+    }
+    w.buf = 0;
+    w.ctl = align256((size_t)2 * w.R * g.nt * 4);
+    w.ctl_bytes = (size_t)(2 + 2 * w.G) * 4;
+    w.total = w.ctl + align256(w.ctl_bytes);
+    return w;
 }
 
 sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v, const int32_t* kept_idx,
@@ -536,7 +560,7 @@ size_t sa_select_workspace_size(const sa_shape* shape, int32_t streamed) {
     Geo g;
     if (geo_of(shape, &g) != SA_OK) return 0;
     if (!streamed) return 0;
-    return select_rows_per_block(g) * (size_t)g.nt * 4;
+    return stream_ws(g).total;
 }
 
 // Short rows: one warp per row, as many rows per CTA as fit in shared memory; long rows:
@@ -594,33 +618,39 @@ static sa_status select_impl(const sa_shape* shape, const float* scores_or_null,
         launch_select(a, (unsigned)g.bh, stream);
         return launch_status();
     }
-    // streamed: score one L2-resident block of rows at a time, then select from it
-    const int64_t R = (int64_t)select_rows_per_block(g);
-    float* blk = static_cast<float*>(workspace_or_null);
-    for (int64_t h = 0; h < g.bh; ++h) {
-        for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
-            const int64_t rows = std::min<int64_t>(R, g.nt - i0);
-            ScoreArgs sc;
-            sc.q_pool = q_pool;
-            sc.k_pool = k_pool;
-            sc.out = blk;
-            sc.ldo = g.nt;
-            sc.nt = (int32_t)g.nt;
-            sc.h0 = (int32_t)h;
-            sc.i0 = (int32_t)i0;
-            sc.rows = (int32_t)rows;
-            launch_scores(sc, 1u, stream);
-            if ((st = launch_status()) != SA_OK) return st;
-            a.scores = blk;
-            a.lds = g.nt;
-            a.h0 = (int32_t)h;
-            a.i0 = (int32_t)i0;
-            a.rows = (int32_t)rows;
-            launch_select(a, 1u, stream);
-            if ((st = launch_status()) != SA_OK) return st;
-        }
+    // streamed: one persistent launch scores blocks of rows into two L2-resident buffers and
+    // selects from them (k_select_stream.cuh)
+    const StreamWs w = stream_ws(g);
+    if (w.items_per_head * g.bh >= (1ll << 31) - 65536 || w.G >= (1ll << 28)) return SA_ERR_UNSUPPORTED;
+    uint8_t* base = static_cast<uint8_t*>(workspace_or_null);
+    StreamSelArgs sa_;
+    sa_.sel = a;
+    sa_.q_pool = q_pool;
+    sa_.k_pool = k_pool;
+    sa_.buf = reinterpret_cast<float*>(base + w.buf);
+    sa_.ctl = reinterpret_cast<int32_t*>(base + w.ctl);
+    sa_.bh = (int32_t)g.bh;
+    sa_.R = (int32_t)w.R;
+    sa_.nblk = (int32_t)w.nblk;
+    sa_.col_tiles = (int32_t)w.col_tiles;
+    sa_.items_per_head = w.items_per_head;
+    sa_.items_total = w.items_per_head * g.bh;
+    const size_t smem = std::max<size_t>(SCORES_BIG_SMEM, select_block_smem_bytes((int)g.nt));
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_stream_kernel, 256, smem) != cudaSuccess ||
+        per_sm < 1) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
     }
-    return SA_OK;
+    if (cudaMemsetAsync(base + w.ctl, 0, w.ctl_bytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    const int64_t grid = std::min<int64_t>((int64_t)sms * per_sm, sa_.items_total);
+    select_stream_kernel<<<(unsigned)std::max<int64_t>(1, grid), 256, smem, stream>>>(sa_);
+    return launch_status();
 }
 
 sa_status sa_select_topk(const sa_shape* shape, const float* scores_or_null, const float* q_pool,
