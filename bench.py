@@ -252,6 +252,13 @@ def attention_work(layer, w):
     return flops, tile_flops
 
 
+def with_frames(w, frames: int):
+    """The workload at another frame count with the same budget k (so the same number of items per
+    query tile, as long as that many candidates exist), under a name that says so."""
+    return w.scaled(name="%s_at%d" % (w.name, frames), frames=frames,
+                    window=min(w.window, frames) if w.window else 0)
+
+
 def dense_flops(w, heads):
     return 4.0 * w.head_dim * heads * float(w.L) * float(w.L)
 
@@ -921,10 +928,14 @@ def main(argv=None):
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
     ap.add_argument("--dense-budget", type=float, default=15.0,
                     help="seconds of timed dense-control calls (at least one call)")
+    ap.add_argument("--frames", type=int, default=0,
+                    help="run the workload at another frame count, same tile sparsity (smaller profiling cases)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = BY_NAME[args.workload]
+    if args.frames:
+        w = with_frames(w, args.frames)
     if args.impl == "reference":
         run_reference(args, w)
     elif args.sga:

@@ -217,9 +217,9 @@ sa_status sa_head_budgets(const sa_shape* shape, const float* q_pool, const floa
 sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, const float* k_pool, int32_t k,
                                  int32_t* kept_idx, int32_t* kept_cnt, int32_t max_kept, sa_stream_t stream);
 
-/* Bytes of workspace sa_sparse_attn_fwd needs: on the tensor-core path (bf16, tile 128) a
- * transposed copy of every V tile it may gather (the size of V plus the sink segment) and, in
- * landmark mode, the bf16 landmark tables; 0 on the CUDA-core path (f32 or tile 64). */
+/* Bytes of workspace sa_sparse_attn_fwd needs: a transposed copy of every V tile it may gather
+ * (the size of V plus the sink segment) and, in landmark mode, the landmark tables, in the
+ * input type; for f32 inputs also Q, K and the sink keys rounded to tf32. */
 size_t sa_sparse_attn_workspace_size(const sa_shape* shape, int32_t landmark);
 
 /*
@@ -235,7 +235,8 @@ size_t sa_sparse_attn_workspace_size(const sa_shape* shape, int32_t landmark);
  * and   O[h][r] = sum_t softmax_t(scale * q_r . k_t + b_t) v_t,
  *       lse[h][r] = ln sum_t exp(scale * q_r . k_t + b_t)       (natural log; optional).
  * O has the shape's dtype, [bh][S*N][d]; lse is f32 [bh][S*N].  Products run on the tensor
- * cores (bf16 in, f32 accumulate; landmark means enter rounded to bf16) with an f32 softmax.
+ * cores with f32 accumulation and an f32 softmax: bf16 operands for bf16 inputs (landmark means
+ * enter rounded to bf16), tf32 operands (each f32 rounded to the nearest tf32) for f32 inputs.
  * Lists must be ascending with entries in [0, nt) and no repeats; a list from sa_select_topk
  * always is.  Entries beyond kept_cnt are ignored.  An out-of-range entry is skipped and
  * reported as SA_ERR_BAD_LIST by sa_check_device_error.
@@ -285,8 +286,8 @@ sa_status sa_sparse_attn_bwd(const sa_shape* shape, const void* q, const void* k
                              void* workspace, size_t workspace_bytes,
                              void* dq, void* dk, void* dv, sa_stream_t stream);
 
-/* Bytes of workspace sa_dense_attn_fwd needs (a transposed copy of V on the tensor-core
- * path, 0 on the CUDA-core path). */
+/* Bytes of workspace sa_dense_attn_fwd needs (a transposed copy of V; for f32 inputs also Q
+ * and K rounded to tf32). */
 size_t sa_dense_attn_workspace_size(const sa_shape* shape);
 
 /*

@@ -93,21 +93,25 @@ def test_workspace_sizes(lib):
     shp = sa.shape(16, 1024, 1374, 64, 128, 5, "bf16")
     assert sa.sa_select_workspace_size(shp, False) == 0
     ws = sa.sa_select_workspace_size(shp, True)
-    # two buffers of R whole score rows (R a multiple of 128, L2-sized together) + control words
-    R = (24 << 20) // (11264 * 4) // 128 * 128
-    nblk = -(-11264 // R)
-    bufs = 2 * R * 11264 * 4
-    assert R == 512 and ws == bufs + -(-(2 + 2 * 16 * nblk) * 4 // 256) * 256
-    assert ws <= 64 << 20
+    assert 0 < ws <= 64 << 20 and ws % (11264 * 4) == 0  # whole score rows, L2-sized
     shp4 = sa.shape(16, 512, 1374, 64, 128, 5, "bf16")
     vt = 16 * 5632 * 64 * 128 * 2                 # transposed V tiles of every key tile
     sinks = 16 * 20 * 64 * 128 * 2                # 512 frames x 5 sinks = 2560 rows = 20 tiles
     assert sa.sa_sparse_attn_workspace_size(shp4, False) == vt + sinks
     assert sa.sa_sparse_attn_workspace_size(shp4, True) >= vt + sinks + 2 * 16 * 5632 * 64 * 2 + 5632 * 4
     assert sa.sa_dense_attn_workspace_size(shp4) == 16 * (-(-512 * 1374 // 128)) * 64 * 128 * 2
-    # the CUDA-core path (f32, or tile 64) needs none
-    assert sa.sa_sparse_attn_workspace_size(sa.shape(2, 4, 256, 64, 64, 0, "f32"), True) == 0
-    assert sa.sa_dense_attn_workspace_size(sa.shape(2, 4, 256, 64, 64, 0, "bf16")) == 0
+    # the 64-key tensor-core path (f32, or tile 64): transposed V in 64-key items of the input type
+    # (f32 also keeps Q, K and the sink keys rounded to tf32)
+    f32_t64 = sa.shape(2, 4, 256, 64, 64, 0, "f32")          # nt 16, no sinks
+    qk = 2 * (2 * 1024 * 64 * 4)
+    assert sa.sa_sparse_attn_workspace_size(f32_t64, False) == 2 * 16 * 64 * 64 * 4 + qk
+    lm = 2 * 16 * 64 * 64 * 4 + 2 * 64 * 64 * 4 + 2 * 64 * 64 * 4 + 256   # + keys, values, bias (ntp 64)
+    assert sa.sa_sparse_attn_workspace_size(f32_t64, True) == lm + qk
+    f32_t128 = sa.shape(1, 3, 300, 64, 128, 5, "f32")       # nt 9, two 64-key items per tile, 15 sinks
+    sk = -(-15 * 64 * 4 // 256) * 256
+    assert sa.sa_sparse_attn_workspace_size(f32_t128, False) == 9 * 2 * 64 * 64 * 4 + 64 * 64 * 4 + \
+        2 * 900 * 64 * 4 + sk
+    assert sa.sa_dense_attn_workspace_size(sa.shape(2, 4, 256, 64, 64, 0, "bf16")) == 2 * 16 * 64 * 64 * 2
 
 
 def test_package_fails_loudly_without_library(tmp_path):

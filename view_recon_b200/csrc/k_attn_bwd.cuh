@@ -824,48 +824,74 @@ __global__ void bwd_scan_lists_kernel(const int32_t* kept_idx, const int32_t* ke
 }
 
 // One block: CSR offsets of the reverse lists (per key tile, over all heads), the unit table
-// (fixed sink / landmark units first, then each key tile's list in runs of kBwdChunk) and the
-// number of units.  fill[] starts at each list's offset for bwd_fill_lists_kernel.
+// and the number of units.  fill[] starts at each list's offset for bwd_fill_lists_kernel.
+// Units are written longest first, so that the persistent dK/dV kernel's round-robin walk over
+// the table gives every CTA about the same work: the fixed sink / landmark units, then every
+// whole run of kBwdChunk query tiles, then the shorter remainders of the lists by length
+// descending (equal lengths in any order: their contributions meet in f32 atomics anyway).
 // Writes at most units_cap units: a plan that would need more (possible only for malformed lists)
 // is cut at the capacity, reported as SA_ERR_BAD_LIST, and the unit count clamped to it.
 __global__ void __launch_bounds__(1024) bwd_plan_kernel(const int32_t* rev_cnt, int32_t* fill, int4* units,
                                                         int32_t* n_units, int32_t bh, int32_t nt,
                                                         int32_t n_sink_tiles, int32_t n_lm_chunks,
                                                         int64_t units_cap) {
-    __shared__ int64_t s_e[1024], s_u[1024];
+    __shared__ int64_t s_e[1024], s_f[1024];
+    __shared__ int32_t s_rem[kBwdChunk];     // remainder units of each length (1 .. kBwdChunk - 1)
+    __shared__ int64_t s_cursor[kBwdChunk];  // next slot of each remainder length
     const int64_t M = (int64_t)bh * nt;
     const int64_t per = (M + 1023) / 1024;
     const int64_t b0 = min(M, per * threadIdx.x), b1 = min(M, b0 + per);
-    int64_t se = 0, su = 0;
+    if (threadIdx.x < kBwdChunk) s_rem[threadIdx.x] = 0;
+    __syncthreads();
+    int64_t se = 0, sf = 0;
     for (int64_t x = b0; x < b1; ++x) {
         const int c = rev_cnt[x];
         se += c;
-        su += (c + kBwdChunk - 1) / kBwdChunk;
+        sf += c / kBwdChunk;
+        if (c % kBwdChunk) atomicAdd(&s_rem[c % kBwdChunk], 1);
     }
     s_e[threadIdx.x] = se;
-    s_u[threadIdx.x] = su;
+    s_f[threadIdx.x] = sf;
     __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {  // inclusive scan (Hillis-Steele)
+    for (int off = 1; off < 1024; off <<= 1) {  // inclusive scans (Hillis-Steele)
         const int64_t ae = threadIdx.x >= off ? s_e[threadIdx.x - off] : 0;
-        const int64_t au = threadIdx.x >= off ? s_u[threadIdx.x - off] : 0;
+        const int64_t af = threadIdx.x >= off ? s_f[threadIdx.x - off] : 0;
         __syncthreads();
         s_e[threadIdx.x] += ae;
-        s_u[threadIdx.x] += au;
+        s_f[threadIdx.x] += af;
         __syncthreads();
     }
     const int64_t chunks_q = (nt + kBwdChunk - 1) / kBwdChunk;
     const int64_t n_fixed = (int64_t)bh * (n_sink_tiles + n_lm_chunks) * chunks_q;
-    int64_t e0 = s_e[threadIdx.x] - se, u0 = n_fixed + s_u[threadIdx.x] - su;
+    const int64_t n_full = s_f[1023];
+    if (threadIdx.x == 0) {  // remainder lengths kBwdChunk-1 down to 1 follow the whole runs
+        int64_t pos = n_fixed + n_full;
+        for (int r = kBwdChunk - 1; r >= 1; --r) {
+            s_cursor[r] = pos;
+            pos += s_rem[r];
+        }
+        s_cursor[0] = pos;  // total
+    }
+    __syncthreads();
+    int64_t e0 = s_e[threadIdx.x] - se, u0 = n_fixed + s_f[threadIdx.x] - sf;
     for (int64_t x = b0; x < b1; ++x) {
         const int c = rev_cnt[x];
         fill[x] = (int32_t)e0;
         const int h = (int)(x / nt), j = (int)(x % nt);
-        for (int q = 0; q * kBwdChunk < c; ++q) {
+        for (int q = 0; (q + 1) * kBwdChunk <= c; ++q) {
             if (u0 >= units_cap) {
                 sa_flag_error(SA_ERR_BAD_LIST);
                 break;
             }
-            units[u0++] = make_int4(h, j, (int32_t)(e0 + q * kBwdChunk), (int32_t)(e0 + min(c, (q + 1) * kBwdChunk)));
+            units[u0++] = make_int4(h, j, (int32_t)(e0 + q * kBwdChunk), (int32_t)(e0 + (q + 1) * kBwdChunk));
+        }
+        const int r = c % kBwdChunk;
+        if (r) {
+            const int64_t slot = (int64_t)atomicAdd(reinterpret_cast<unsigned long long*>(&s_cursor[r]), 1ull);
+            if (slot >= units_cap)
+                sa_flag_error(SA_ERR_BAD_LIST);
+            else
+                units[slot] = make_int4(h, j, (int32_t)(e0 + c - r), (int32_t)(e0 + c));
         }
         e0 += c;
     }
@@ -878,7 +904,7 @@ __global__ void __launch_bounds__(1024) bwd_plan_kernel(const int32_t* rev_cnt, 
         const int item = it < n_sink_tiles ? it : it - n_sink_tiles;
         units[f] = make_int4(h, (kind << 24) | item, q * kBwdChunk, min(nt, (q + 1) * kBwdChunk));
     }
-    if (threadIdx.x == 1023) *n_units = (int32_t)min(units_cap, n_fixed + s_u[1023]);
+    if (threadIdx.x == 1023) *n_units = (int32_t)min(units_cap, s_cursor[0]);
 }
 
 __global__ void bwd_fill_lists_kernel(const int32_t* kept_idx, const int32_t* kept_cnt, int32_t max_kept,

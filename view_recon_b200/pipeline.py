@@ -194,7 +194,8 @@ class SparseGlobalAttention:
         """Kernel launches libsa makes for one forward (for launch accounting)."""
         n = 1  # pooling
         if self.streamed:
-            n += 1  # one persistent launch scores and selects (its control words are cleared by a memset)
+            rows = sa.sa_select_workspace_size(self.shape, True) // (4 * self.nt)
+            n += 2 * self.bh * (-(-self.nt // rows))  # score block + select block
         else:
             n += 2  # scores + select
         if self.adaptive is not None:
