@@ -1,8 +1,8 @@
 // Step 1: tile pooling ("Zebra3D" abstract: tile summaries; "AVGGT" 2.B.2: mean key/value).
 //
-// One warp per (head, tile).  A tile's rows are contiguous in memory, so the warp streams
-// [first row, last row) with 128-bit read-only loads, 512 contiguous bytes per instruction
-// for bf16 (4 rows of 64 elements), accumulates in f32 registers and reduces with shuffles.
+// A tile's rows are contiguous in memory and are streamed with 128-bit read-only loads, 512
+// contiguous bytes per warp instruction for bf16 (4 rows of 64 elements), accumulated in f32
+// registers and reduced with shuffles (bf16: four warps per tile; f32: one warp per tile).
 // HBM bound: every byte of Q and K (and V in landmark mode) is read exactly once.
 #pragma once
 #include "sa_device.cuh"
@@ -29,47 +29,40 @@ __device__ __forceinline__ void bf16x8_accum(const uint4& u, float (&acc)[8]) {
     }
 }
 
-// d = 64, bf16: lane = (row group r4 in 0..3, 16-byte chunk c in 0..7).
-__global__ void __launch_bounds__(256) pool_tiles_bf16_kernel(PoolArgs a) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (warp >= a.bh * a.nt) return;
-    const int h = warp / a.nt, j = warp % a.nt;
+// d = 64, bf16: one 128-thread CTA per (head, tile).  Warp w sums rows [w*T/4, (w+1)*T/4) of the
+// tile, lane = (row group r4 in 0..3, 16-byte chunk c in 0..7), every load of its rows in flight at
+// once (8 per tensor at T = 128); the four warps' partial sums meet in shared memory and are added
+// in warp order (deterministic).
+__global__ void __launch_bounds__(128) pool_tiles_bf16_kernel(PoolArgs a) {
+    __shared__ float part[3][4][64];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y, j = blockIdx.x;
     const int f = j / a.tpf, slot = j % a.tpf;
     const int n0 = slot * a.tile;
     const int nq = min(a.tile, a.tokens - n0);
     const int lo = min(nq, max(0, a.n_sink - n0));  // first key row inside the tile
     const int64_t row0 = (int64_t)h * a.frames * a.tokens + (int64_t)f * a.tokens + n0;
     const int c = lane & 7, r4 = lane >> 3;
+    const int per_warp = a.tile / 4;  // 32 or 16 rows
+    const int rw0 = warp * per_warp;
     const uint4* q4 = reinterpret_cast<const uint4*>(a.q) + row0 * 8 + c;
     const uint4* k4 = reinterpret_cast<const uint4*>(a.k) + row0 * 8 + c;
     const uint4* v4 = a.v_pool ? reinterpret_cast<const uint4*>(a.v) + row0 * 8 + c : nullptr;
-
     float sq[8] = {}, sk[8] = {}, sv[8] = {};
-    int r = r4;
-    for (; r + 12 < nq; r += 16) {  // 4 rows per lane in flight per tensor
-        uint4 uq[4], uk[4], uv[4];
+    uint4 uq[8], uk[8], uv[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            uq[u] = __ldg(q4 + (int64_t)(r + 4 * u) * 8);
-            uk[u] = __ldg(k4 + (int64_t)(r + 4 * u) * 8);
-            if (v4) uv[u] = __ldg(v4 + (int64_t)(r + 4 * u) * 8);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            bf16x8_accum(uq[u], sq);
-            if (r + 4 * u >= lo) {
-                bf16x8_accum(uk[u], sk);
-                if (v4) bf16x8_accum(uv[u], sv);
-            }
-        }
+    for (int u = 0; u < 8; ++u) {
+        const int r = rw0 + r4 + 4 * u;
+        const bool in = 4 * u < per_warp && r < nq;
+        uq[u] = in ? __ldg(q4 + (int64_t)r * 8) : make_uint4(0, 0, 0, 0);
+        uk[u] = (in && r >= lo) ? __ldg(k4 + (int64_t)r * 8) : make_uint4(0, 0, 0, 0);
+        uv[u] = (v4 && in && r >= lo) ? __ldg(v4 + (int64_t)r * 8) : make_uint4(0, 0, 0, 0);
     }
-    for (; r < nq; r += 4) {
-        bf16x8_accum(__ldg(q4 + (int64_t)r * 8), sq);
-        if (r >= lo) {
-            bf16x8_accum(__ldg(k4 + (int64_t)r * 8), sk);
-            if (v4) bf16x8_accum(__ldg(v4 + (int64_t)r * 8), sv);
-        }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        bf16x8_accum(uq[u], sq);
+        bf16x8_accum(uk[u], sk);
+        if (v4) bf16x8_accum(uv[u], sv);
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -80,27 +73,30 @@ __global__ void __launch_bounds__(256) pool_tiles_bf16_kernel(PoolArgs a) {
         sv[e] += __shfl_xor_sync(0xffffffffu, sv[e], 8);
         sv[e] += __shfl_xor_sync(0xffffffffu, sv[e], 16);
     }
-    const int nk = nq - lo;
     if (lane < 8) {
-        const float iq = 1.0f / (float)nq;
-        const float ik = nk > 0 ? 1.0f / (float)nk : 0.0f;
-        float4* qp = reinterpret_cast<float4*>(a.q_pool + ((int64_t)h * a.nt + j) * 64 + 8 * c);
-        float4* kp = reinterpret_cast<float4*>(a.k_pool + ((int64_t)h * a.nt + j) * 64 + 8 * c);
-        qp[0] = make_float4(sq[0] * iq, sq[1] * iq, sq[2] * iq, sq[3] * iq);
-        qp[1] = make_float4(sq[4] * iq, sq[5] * iq, sq[6] * iq, sq[7] * iq);
-        kp[0] = make_float4(sk[0] * ik, sk[1] * ik, sk[2] * ik, sk[3] * ik);
-        kp[1] = make_float4(sk[4] * ik, sk[5] * ik, sk[6] * ik, sk[7] * ik);
-        if (a.v_pool) {
-            float4* vp = reinterpret_cast<float4*>(a.v_pool + ((int64_t)h * a.nt + j) * 64 + 8 * c);
-            vp[0] = make_float4(sv[0] * ik, sv[1] * ik, sv[2] * ik, sv[3] * ik);
-            vp[1] = make_float4(sv[4] * ik, sv[5] * ik, sv[6] * ik, sv[7] * ik);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            part[0][warp][8 * c + e] = sq[e];
+            part[1][warp][8 * c + e] = sk[e];
+            part[2][warp][8 * c + e] = sv[e];
         }
     }
-    if (h == 0 && lane == 0) a.k_cnt[j] = nk;
+    __syncthreads();
+    const int nk = nq - lo;
+    if (threadIdx.x < 64) {
+        const int d = threadIdx.x;
+        const float iq = 1.0f / (float)nq;
+        const float ik = nk > 0 ? 1.0f / (float)nk : 0.0f;
+        const int64_t o = ((int64_t)h * a.nt + j) * 64 + d;
+        a.q_pool[o] = (((part[0][0][d] + part[0][1][d]) + part[0][2][d]) + part[0][3][d]) * iq;
+        a.k_pool[o] = (((part[1][0][d] + part[1][1][d]) + part[1][2][d]) + part[1][3][d]) * ik;
+        if (a.v_pool) a.v_pool[o] = (((part[2][0][d] + part[2][1][d]) + part[2][2][d]) + part[2][3][d]) * ik;
+    }
+    if (h == 0 && threadIdx.x == 0) a.k_cnt[j] = nk;
     // sink rows of this tile (only tiles that start before n_sink hold any)
     if (lo > 0 && a.sink_k) {
         const int64_t srow0 = (int64_t)h * a.frames * a.n_sink + (int64_t)f * a.n_sink + n0;
-        for (int idx = lane; idx < lo * 8; idx += 32) {
+        for (int idx = threadIdx.x; idx < lo * 8; idx += 128) {
             const int rr = idx >> 3, cc = idx & 7;
             reinterpret_cast<uint4*>(a.sink_k)[(srow0 + rr) * 8 + cc] =
                 __ldg(reinterpret_cast<const uint4*>(a.k) + (row0 + rr) * 8 + cc);

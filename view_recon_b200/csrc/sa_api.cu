@@ -616,9 +616,9 @@ sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, cons
     a.nt = (int32_t)g.nt;
     const int64_t warps = g.bh * g.nt;
     const int64_t blocks = (warps + 7) / 8;
-    if (blocks >= (int64_t(1) << 31)) return SA_ERR_UNSUPPORTED;
+    if (blocks >= (int64_t(1) << 31) || g.bh > 65535 || g.nt >= (int64_t(1) << 31)) return SA_ERR_UNSUPPORTED;
     if (g.bf16)
-        pool_tiles_bf16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+        pool_tiles_bf16_kernel<<<dim3((unsigned)g.nt, (unsigned)g.bh), 128, 0, stream>>>(a);
     else
         pool_tiles_f32_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
     return launch_status();
