@@ -464,6 +464,36 @@ def time_layer(w, q, k, v, dev, steps: int, warmup: int, flush, clocks=None):
     return layer, stage, clk
 
 
+def time_graph(layer, q, k, v, dev, steps: int, warmup: int, flush) -> float:
+    """Mean ms of one layer call replayed from a CUDA graph (the same launches as the eager call,
+    recorded once by `SparseGlobalAttention.capture`), L2 flushed before every replay, CUDA
+    events on the replaying stream."""
+    import torch
+    from view_recon_b200 import sa
+    g = layer.capture(q, k, v)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        flush()
+        g.replay()
+    torch.cuda.synchronize(dev)
+    dist_barrier(dev)
+    evs = []
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    dist_barrier(dev)
+    status = sa.sa_check_device_error()
+    if status != 0:
+        raise RuntimeError("device error in graph replays: %s" % sa.status_string(status))
+    del g
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
 def time_dense(w, q, k, v, dev, flush, budget_s: float = 20.0):
     """Dense control at the same shape: one untimed call, then as many timed calls as fit the
     budget (at least one, at most ten).  Returns mean ms per call."""
@@ -505,9 +535,11 @@ def side_config(wname: str, dev, steps: int, warmup: int, flush) -> dict:
     flops, tile_flops = attention_work(layer, w)
     peak, peak_desc, burst = tensor_peak(ms_attn)
     achieved = flops / (ms_attn / 1e3) / 1e12
+    graph_ms = time_graph(layer, q, k, v, dev, steps, warmup, flush)
     del layer
     dense_ms, n_dense = time_dense(w, q, k, v, dev, flush, budget_s=6.0)
     out = {"tokens_per_s": w.L / (total / 1e3), "ms_per_call": total, "steps": steps,
+           "graph_ms_per_call": graph_ms,
            "stages_ms": {"pool": ms_pool, "score": ms_score, "select": ms_select, "attn": ms_attn},
            "attn_tflops_algorithmic": achieved, "attn_tflops_kept_tiles": tile_flops / (ms_attn / 1e3) / 1e12,
            "frac": achieved / peak, "frac_of_burst": achieved / burst, "peak": peak, "peak_source": peak_desc,
@@ -556,6 +588,8 @@ def run_ours(args, w):
     flops, tile_flops = attention_work(layer, w)
     per_step = layer.launches_per_call()
     max_kept = layer.max_kept
+    # the same call replayed from one CUDA graph
+    graph_ms = dist_max(time_graph(layer, q, k, v, dev, args.steps, args.warmup, flush), dev)
     del layer
     torch.cuda.empty_cache()
 
@@ -609,6 +643,8 @@ def run_ours(args, w):
         "data": "synthetic latent-point Q/K/V (seeded; no dataset or weights)",
         "config": run_config(w_job, w, world, sharded),
         "stages_ms": {"pool": ms_pool, "score": ms_score, "select": ms_select, "attn": ms_attn},
+        "graph": {"ms_per_call": graph_ms, "tokens_per_s": whole_job_rate(w.L * calls_here, world, 1, graph_ms),
+                  "note": "the same call replayed from one CUDA graph (capture once, replay per step)"},
         "attn_tflops_algorithmic": achieved,
         "attn_tflops_kept_tiles": tile_flops / (ms_attn / 1e3) / 1e12,
         "attn_only_tokens_per_s": w.L / (ms_attn / 1e3),

@@ -157,6 +157,23 @@ class SparseGlobalAttention:
 
     __call__ = forward
 
+    def capture(self, q, k, v):
+        """Record one whole layer call on these input tensors as a CUDA graph and return it.
+
+        `g.replay()` then re-runs every launch of the call (pooling, scoring, selection -- a few
+        hundred launches in streamed mode -- and attention) from one host call, on the current
+        stream; new inputs are written into q, k, v in place before a replay, and the results
+        land in `self.buf.o` / `self.buf.lse` as with `forward`.  The library allocates nothing
+        and every step is stream-ordered, so the call is captured as it runs.  One eager call
+        comes first so that no kernel attribute is set inside the capture."""
+        import torch
+        self.forward(q, k, v)
+        torch.cuda.current_stream(self.device).synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.forward(q, k, v)
+        return g
+
     def backward(self, q, k, v, d_o, stream=None):
         """Gradients (dq, dk, dv) of sum(d_o * O) for the last forward on these q, k, v, with its
         kept lists held fixed; d_o is [bh][S*N][d] like O.  Needs the forward's LSE."""
