@@ -12,6 +12,7 @@
 #include "k_budget.cuh"
 #include "k_pool.cuh"
 #include "k_scores.cuh"
+#include "k_scores_tc.cuh"
 #include "k_select.cuh"
 #include "k_sga.cuh"
 
@@ -108,6 +109,8 @@ sa_status ensure_attributes() {
                                (int)bw::KVLay::smem_bytes()) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tile_scores_big_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SCORES_BIG_SMEM) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)stc::kSmemBytes) == cudaSuccess;
     ok &= cudaFuncSetAttribute(head_stat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BUDGET_SMEM) ==
           cudaSuccess;
     ok &= cudaFuncSetAttribute(select_topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -624,6 +627,46 @@ sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, cons
     return launch_status();
 }
 
+#ifndef SA_SCORES_TC
+#define SA_SCORES_TC 1
+#endif
+
+// Step 2 on the tensor cores (k_scores_tc.cuh): the pooled tables' tensor maps are encoded once
+// per call; each launch then covers rows [i0, i0 + rows) of heads h0 .. h0 + gz - 1.
+struct ScoreTcLaunch {
+    ScoreTcArgs a;
+};
+
+static bool score_tc_prepare(ScoreTcLaunch* L, const Geo& g, const float* q_pool, const float* k_pool, float* out,
+                             int64_t ldo) {
+    memset(&L->a, 0, sizeof(L->a));
+    if (!encode_rows_e(&L->a.tm_q, q_pool, g.bh * g.nt, false, 128) ||
+        !encode_rows_e(&L->a.tm_k, k_pool, g.bh * g.nt, false, 128))
+        return false;
+    L->a.out = out;
+    L->a.ldo = ldo;
+    L->a.nt = (int32_t)g.nt;
+    L->a.n_chunks = (int32_t)((g.nt + 127) / 128);
+    L->a.vec_out = (ldo % 4 == 0 && aligned16(out)) ? 1 : 0;
+    return true;
+}
+
+static sa_status score_tc_launch(ScoreTcLaunch* L, int64_t h0, int64_t i0, int64_t rows, int64_t gz,
+                                 cudaStream_t stream) {
+    ScoreTcArgs& a = L->a;
+    a.h0 = (int32_t)h0;
+    a.i0 = (int32_t)i0;
+    a.rows = (int32_t)rows;
+    const int64_t gy = (rows + 127) / 128;
+    if (gy > 65535 || gz > 65535 || gy < 1 || gz < 1) return SA_ERR_UNSUPPORTED;
+    // at least two CTAs per SM (148 SMs) where the chunks allow it: one CTA (192 KB) per SM at a time
+    const int64_t want_x = std::max<int64_t>(1, std::min<int64_t>(a.n_chunks, (2 * 148 + gy * gz - 1) / (gy * gz)));
+    a.chunks_per_cta = (int32_t)((a.n_chunks + want_x - 1) / want_x);
+    const int64_t gx = (a.n_chunks + a.chunks_per_cta - 1) / a.chunks_per_cta;
+    score_tc_kernel<<<dim3((unsigned)gx, (unsigned)gy, (unsigned)gz), 384, stc::kSmemBytes, stream>>>(a);
+    return launch_status();
+}
+
 // Large tile counts: 128 x 128 blocks (8 x 8 outputs per thread); small ones keep 64 x 64 blocks
 // so that enough CTAs fill the GPU.
 static void launch_scores(const ScoreArgs& a, unsigned gz, cudaStream_t stream) {
@@ -655,6 +698,11 @@ sa_status sa_tile_scores(const sa_shape* shape, const float* q_pool, const float
     a.rows = (int32_t)g.nt;
     if ((g.nt + 63) / 64 > 65535) return SA_ERR_UNSUPPORTED;
     if ((st = ensure_attributes()) != SA_OK) return st;
+    if (SA_SCORES_TC) {
+        ScoreTcLaunch L;
+        if (!score_tc_prepare(&L, g, q_pool, k_pool, scores, g.nt)) return SA_ERR_CUDA;
+        return score_tc_launch(&L, 0, 0, g.nt, g.bh, stream);
+    }
     launch_scores(a, (unsigned)g.bh, stream);
     return launch_status();
 }
@@ -726,20 +774,26 @@ static sa_status select_impl(const sa_shape* shape, const float* scores_or_null,
     // measured slower: 23.9 ms against 17.9 ms at 1024 frames)
     const int64_t R = (int64_t)select_rows_per_block(g);
     float* blk = static_cast<float*>(workspace_or_null);
+    ScoreTcLaunch L;
+    if (SA_SCORES_TC && !score_tc_prepare(&L, g, q_pool, k_pool, blk, g.nt)) return SA_ERR_CUDA;
     for (int64_t h = 0; h < g.bh; ++h) {
         for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
             const int64_t rows = std::min<int64_t>(R, g.nt - i0);
-            ScoreArgs sc;
-            sc.q_pool = q_pool;
-            sc.k_pool = k_pool;
-            sc.out = blk;
-            sc.ldo = g.nt;
-            sc.nt = (int32_t)g.nt;
-            sc.h0 = (int32_t)h;
-            sc.i0 = (int32_t)i0;
-            sc.rows = (int32_t)rows;
-            launch_scores(sc, 1u, stream);
-            if ((st = launch_status()) != SA_OK) return st;
+            if (SA_SCORES_TC) {
+                if ((st = score_tc_launch(&L, h, i0, rows, 1, stream)) != SA_OK) return st;
+            } else {
+                ScoreArgs sc;
+                sc.q_pool = q_pool;
+                sc.k_pool = k_pool;
+                sc.out = blk;
+                sc.ldo = g.nt;
+                sc.nt = (int32_t)g.nt;
+                sc.h0 = (int32_t)h;
+                sc.i0 = (int32_t)i0;
+                sc.rows = (int32_t)rows;
+                launch_scores(sc, 1u, stream);
+                if ((st = launch_status()) != SA_OK) return st;
+            }
             a.scores = blk;
             a.lds = g.nt;
             a.h0 = (int32_t)h;
@@ -794,20 +848,26 @@ sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, con
     a.max_kept = max_kept;
     a.k_head = nullptr;
     a.k_max = k;
+    ScoreTcLaunch L;
+    if (SA_SCORES_TC && !score_tc_prepare(&L, g, q_pool, k_pool, blk, g.nt)) return SA_ERR_CUDA;
     for (int64_t h = 0; h < g.bh; ++h) {
         for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
             const int64_t rows = std::min<int64_t>(R, g.nt - i0);
-            ScoreArgs sc;
-            sc.q_pool = q_pool;
-            sc.k_pool = k_pool;
-            sc.out = blk;
-            sc.ldo = g.nt;
-            sc.nt = (int32_t)g.nt;
-            sc.h0 = (int32_t)h;
-            sc.i0 = (int32_t)i0;
-            sc.rows = (int32_t)rows;
-            launch_scores(sc, 1u, stream);
-            if ((st = launch_status()) != SA_OK) return st;
+            if (SA_SCORES_TC) {
+                if ((st = score_tc_launch(&L, h, i0, rows, 1, stream)) != SA_OK) return st;
+            } else {
+                ScoreArgs sc;
+                sc.q_pool = q_pool;
+                sc.k_pool = k_pool;
+                sc.out = blk;
+                sc.ldo = g.nt;
+                sc.nt = (int32_t)g.nt;
+                sc.h0 = (int32_t)h;
+                sc.i0 = (int32_t)i0;
+                sc.rows = (int32_t)rows;
+                launch_scores(sc, 1u, stream);
+                if ((st = launch_status()) != SA_OK) return st;
+            }
             a.scores = blk;
             a.lds = g.nt;
             a.h0 = (int32_t)h;
