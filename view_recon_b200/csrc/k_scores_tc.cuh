@@ -16,8 +16,9 @@
 //   warpgroup 1      splits the landed f32 operands in place into hi (same buffer) and lo (the
 //                    buffer 32 KB above it); the split is elementwise, so the swizzled layout
 //                    carries over to the lo buffer unchanged;
-//   warpgroup 2      epilogue: thread r loads row r of the chunk (128 columns) from TMEM and
-//                    stores the valid columns of its row.
+//   warpgroup 2      epilogue: thread r loads row r of the chunk (128 columns) from TMEM; each
+//                    warp then passes its 32 rows through shared memory 32 columns at a time, so
+//                    that every store instruction writes whole 128-byte runs of a row.
 // TMEM: two 128-column accumulators, so the epilogue of one chunk overlaps the next chunk's MMAs.
 // Every wait is bounded (g_sa_wait_limit_ns) and drains what the role has in flight.
 #pragma once
@@ -41,7 +42,9 @@ constexpr int kAtomBytes = 128 * 128;          // 128 rows x 32 f32
 constexpr int kTileBytes = 2 * kAtomBytes;     // 128 rows x 64 f32
 constexpr int kA = 0;                          // A hi, then A lo
 constexpr int kB = 2 * kTileBytes;             // [2 stages] B hi, then B lo
-constexpr int kBars = kB + 2 * 2 * kTileBytes;
+constexpr int kStage = kB + 2 * 2 * kTileBytes;  // epilogue staging: [4 warps][32 rows][36] f32
+constexpr int kStageRow = 36;                      // floats per staged row (16-byte aligned, conflict-free)
+constexpr int kBars = kStage + 4 * 32 * kStageRow * 4;
 // a_full, a_ready, b_full[2], b_ready[2], b_empty[2], d_full[2], d_empty[2], drain
 constexpr int kNumBars = 13;
 constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, abort flag
@@ -82,18 +85,31 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
-// 32 consecutive scores of one row: 16-byte stores when the whole chunk is valid and aligned,
-// else the first `valid` one by one.
-__device__ __forceinline__ void store_part(float* dst, const uint32_t (&v)[32], int valid, bool vec) {
+// One 32 x 32 piece of a warp's rows (row = lane's TMEM lane, 32 columns from column c0 of
+// the launch's output rows): staged in the warp's shared buffer, then stored row by row.
+// vec: 16-byte stores (8 lanes per row, 4 rows per instruction); else one float per lane.
+__device__ __forceinline__ void store_piece(float* st, const uint32_t (&v)[32], float* out, int64_t ldo,
+                                            int row0, int rows_valid, int c0, int cols_valid, bool vec, int lane) {
+    float4* mine = reinterpret_cast<float4*>(st + lane * kStageRow);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+        mine[u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]), __uint_as_float(v[4 * u + 2]),
+                              __uint_as_float(v[4 * u + 3]));
+    __syncwarp();
     if (vec) {
+        const int rr = lane >> 3, cc = 4 * (lane & 7);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            reinterpret_cast<uint4*>(dst)[u] = make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        for (int j = 0; j < 8; ++j) {
+            const int r = 4 * j + rr;
+            if (row0 + r < rows_valid)
+                *reinterpret_cast<float4*>(out + (int64_t)(row0 + r) * ldo + c0 + cc) =
+                    *reinterpret_cast<const float4*>(st + r * kStageRow + cc);
+        }
     } else {
-#pragma unroll
-        for (int u = 0; u < 32; ++u)
-            if (u < valid) dst[u] = __uint_as_float(v[u]);
+        for (int r = 0; r < 32; ++r)
+            if (row0 + r < rows_valid && lane < cols_valid) out[(int64_t)(row0 + r) * ldo + c0 + lane] = st[r * kStageRow + lane];
     }
+    __syncwarp();
 }
 
 }  // namespace stc
@@ -236,11 +252,9 @@ __global__ void __launch_bounds__(384, 1) score_tc_kernel(const __grid_constant_
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------------ epilogue
-        const int quad = warp & 3;
-        const int r = quad * 32 + lane;          // row of the tile = TMEM lane
-        const int lr = r0 + r;                   // local row of the launch
-        const bool row_ok = lr < a.rows;
-        float* orow = a.out + ((int64_t)blockIdx.z * a.rows + (row_ok ? lr : 0)) * a.ldo;
+        const int quad = warp & 3;               // rows quad*32 .. +31 of the tile = its TMEM lanes
+        float* out_z = a.out + (int64_t)blockIdx.z * a.rows * a.ldo;  // row 0 of this head's rows
+        float* st = reinterpret_cast<float*>(smem + kStage) + quad * 32 * kStageRow;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         bool ok = true;
         for (int n = 0; n < n_chunks && ok; ++n) {
@@ -260,15 +274,14 @@ __global__ void __launch_bounds__(384, 1) score_tc_kernel(const __grid_constant_
             reg_fence(v3);
             tc_fence_before();
             mbar_arrive(&d_empty[s]);  // the accumulator may be overwritten from here on
-            if (!row_ok) continue;
             const int c0 = (c_begin + n) * 128;
             const int valid = min(128, a.nt - c0);
-            float* dst = orow + c0;
             const bool vec = a.vec_out && valid == 128;
-            stc::store_part(dst, v0, valid, vec);
-            stc::store_part(dst + 32, v1, valid - 32, vec);
-            stc::store_part(dst + 64, v2, valid - 64, vec);
-            stc::store_part(dst + 96, v3, valid - 96, vec);
+            const int row0 = r0 + quad * 32;  // first local row of this warp
+            stc::store_piece(st, v0, out_z, a.ldo, row0, a.rows, c0, valid, vec, lane);
+            stc::store_piece(st, v1, out_z, a.ldo, row0, a.rows, c0 + 32, valid - 32, vec, lane);
+            stc::store_piece(st, v2, out_z, a.ldo, row0, a.rows, c0 + 64, valid - 64, vec, lane);
+            stc::store_piece(st, v3, out_z, a.ldo, row0, a.rows, c0 + 96, valid - 96, vec, lane);
         }
     }
 

@@ -659,9 +659,12 @@ static sa_status score_tc_launch(ScoreTcLaunch* L, int64_t h0, int64_t i0, int64
     a.rows = (int32_t)rows;
     const int64_t gy = (rows + 127) / 128;
     if (gy > 65535 || gz > 65535 || gy < 1 || gz < 1) return SA_ERR_UNSUPPORTED;
-    // at least two CTAs per SM (148 SMs) where the chunks allow it: one CTA (192 KB) per SM at a time
-    const int64_t want_x = std::max<int64_t>(1, std::min<int64_t>(a.n_chunks, (2 * 148 + gy * gz - 1) / (gy * gz)));
-    a.chunks_per_cta = (int32_t)((a.n_chunks + want_x - 1) / want_x);
+    // One CTA per SM at a time (211 KB of shared memory): with fewer row tiles than SMs the chunks
+    // of a row tile are split so that the grid is one wave of at most 148 CTAs; otherwise every
+    // CTA takes whole row tiles.
+    const int64_t tiles = gy * gz;
+    const int64_t per_tile = tiles >= 148 ? 1 : 148 / tiles;
+    a.chunks_per_cta = (int32_t)((a.n_chunks + per_tile - 1) / per_tile);
     const int64_t gx = (a.n_chunks + a.chunks_per_cta - 1) / a.chunks_per_cta;
     score_tc_kernel<<<dim3((unsigned)gx, (unsigned)gy, (unsigned)gz), 384, stc::kSmemBytes, stream>>>(a);
     return launch_status();
