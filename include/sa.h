@@ -115,7 +115,11 @@ sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, cons
  *
  *   scores[h][i][j] = sum_e q_pool[h][i][e] * k_pool[h][j][e]     (f32 [bh][nt][nt])
  *
- * Exact f32 dot products (SIMT FMA, e ascending).  No 1/sqrt(d): it does not change a ranking.
+ * f32-accurate dot products on the tensor cores: each f32 operand is split into two tf32 parts
+ * (hi = x rounded to tf32, lo = x - hi rounded to tf32) and hi.hi + hi.lo + lo.hi is accumulated
+ * in f32; the error stays below about 2^-21 * sum_e |q_e k_e|.  No 1/sqrt(d): it does not change
+ * a ranking.  q_pool, k_pool and scores 16-byte aligned; rows of nt scores (a row length that is a
+ * multiple of 4 gets 16-byte stores).
  */
 sa_status sa_tile_scores(const sa_shape* shape, const float* q_pool, const float* k_pool,
                          float* scores, sa_stream_t stream);

@@ -1,8 +1,9 @@
 """Tile scores on the GPU against an fp64 product, element by element.
 
 The bound is the fp32 accumulation bound used throughout: |gpu - fp64| <= 1e-5 * sum_e |q_e k_e| + 1e-9.
-Tile counts cover both kernels (64 x 64 blocks below 1024 tiles, 128 x 128 blocks above) and
-ragged edges: not a multiple of 64, of 128 or of 4.
+The kernel splits every f32 operand into two tf32 parts and sums three tf32 products, which stays
+well inside it (about 2^-21 of sum_e |q_e k_e|).  Tile counts cover one and many 128-column chunks
+per CTA and ragged edges: not a multiple of 64, of 128 or of 4 (scalar rather than 16-byte stores).
 """
 import numpy as np
 import pytest

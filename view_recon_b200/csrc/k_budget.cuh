@@ -7,8 +7,7 @@
 //     k_h = min(k_hi, max(k_lo, floor(beta * P_h + 1/2))).
 //
 // head_stat_kernel: one 256-thread CTA per (128 query tiles, head) walks every 128-column block
-// of key tiles.  The scores come from the same f32 FMA chain as the score kernels (e ascending),
-// in 8 x 8 register blocks; each thread keeps, for its 8 rows, the running triple
+// of key tiles.  The scores are f32 FMA chains over e ascending, in 8 x 8 register blocks; each thread keeps, for its 8 rows, the running triple
 //     m = max x,  Z = sum exp(x - m),  A = sum (x - m) exp(x - m)        (x = temperature * s)
 // so that H = ln Z - A / Z without a second pass.  The 16 threads sharing a row merge their
 // triples in a fixed order and the row's perplexity exp(H) lands in the workspace.

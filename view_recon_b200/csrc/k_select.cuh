@@ -385,7 +385,7 @@ __device__ __forceinline__ bool select_row_block(const SelectArgs& a, int h, int
     __shared__ uint32_t list_n;
     __shared__ int abort_flag;
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int f0 = (i / a.tpf) * a.tpf, f1 = f0 + a.tpf;  // own-frame tiles [f0, f1)
     const int s0 = a.n_sink / a.tile;                      // slots below s0 hold no key row
 
@@ -461,28 +461,52 @@ __device__ __forceinline__ bool select_row_block(const SelectArgs& a, int h, int
 
     // ---- 2. bitmask of tiles above the boundary bin; list of the tiles inside it (the list
     // overwrites hist1, whose last reads precede the syncs inside sel_find_bin)
-    for (int wd = warp; wd < nwords; wd += SEL_BLOCK_THREADS / 32) {
-        const int c = wd * 32 + lane;
-        const uint32_t key = c < nt ? keys[c] : 0u;
-        const bool own = c >= f0 && c < f1;
-        bool sel, in = false;
-        if (mode == 0) {
-            sel = own;
-        } else if (mode == 1) {
-            sel = own || key != 0u;
-        } else {
-            const uint32_t top = key >> 20;
-            sel = own || (key != 0u && (top > prefix || (whole && top == prefix)));
-            in = !whole && key != 0u && top == prefix;
+    // One thread per 32-tile word builds both masks in registers: selected = key at or above
+    // sel_from (candidates only: key >= 1), boundary = key in [in_lo, in_lo + in_span).  Thread
+    // t reads the word's keys starting at element t mod 32, so that a warp's shared-memory
+    // reads hit 32 different banks.
+    {
+        uint32_t sel_from = 0xFFFFFFFFu, in_lo = 0u, in_span = 0u;
+        bool sel_none = mode == 0;
+        if (mode == 1) {
+            sel_from = 1u;
+        } else if (mode == 2) {
+            const uint32_t lo = prefix << 20;
+            if (whole) {
+                sel_from = max(lo, 1u);
+            } else {
+                sel_from = prefix == 0xFFFu ? 0xFFFFFFFFu : (prefix + 1u) << 20;
+                sel_none = prefix == 0xFFFu;  // nothing lies above the top bin
+                in_lo = lo;
+                in_span = 1u << 20;
+            }
         }
-        const uint32_t bs = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) selmask[wd] = bs;
-        const uint32_t bi = __ballot_sync(0xffffffffu, in);
-        if (bi) {
-            uint32_t base = 0;
-            if (lane == 0) base = atomicAdd(&list_n, (uint32_t)__popc(bi));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (in) lst[base + __popc(bi & ((1u << lane) - 1u))] = (uint16_t)c;
+        for (int wd = tid; wd < nwords; wd += SEL_BLOCK_THREADS) {
+            uint32_t sm = 0u, im = 0u;
+#pragma unroll 8
+            for (int j = 0; j < 32; ++j) {
+                const int jj = (j + wd) & 31;
+                const uint32_t key = keys[wd * 32 + jj];  // past nt: slack or the next region, masked below
+                const uint32_t sbit = (!sel_none && key >= sel_from && key != 0u) ? 1u : 0u;
+                const uint32_t ibit = (key != 0u && key - in_lo < in_span) ? 1u : 0u;
+                sm |= sbit << jj;
+                im |= ibit << jj;
+            }
+            const int rem = nt - wd * 32;  // valid tiles in this word
+            const uint32_t valid = rem >= 32 ? 0xFFFFFFFFu : ((1u << rem) - 1u);
+            const int lo = min(max(f0 - 32 * wd, 0), 32), hi = min(max(f1 - 32 * wd, 0), 32);
+            const uint32_t own = (hi == 32 ? 0xFFFFFFFFu : ((1u << hi) - 1u)) & ~(lo == 32 ? 0xFFFFFFFFu : ((1u << lo) - 1u));
+            sm = (sm & valid) | own;
+            im &= valid & ~own;
+            selmask[wd] = sm;
+            if (im) {
+                uint32_t base = atomicAdd(&list_n, (uint32_t)__popc(im));
+                while (im) {
+                    const int b = __ffs(im) - 1;
+                    im &= im - 1u;
+                    lst[base++] = (uint16_t)(wd * 32 + b);
+                }
+            }
         }
     }
     __syncthreads();

@@ -11,7 +11,6 @@
 #include "k_attn_tcg.cuh"
 #include "k_budget.cuh"
 #include "k_pool.cuh"
-#include "k_scores.cuh"
 #include "k_scores_tc.cuh"
 #include "k_select.cuh"
 #include "k_sga.cuh"
@@ -107,8 +106,6 @@ sa_status ensure_attributes() {
                                (int)bw::QLay::smem_bytes()) == cudaSuccess;
     ok &= cudaFuncSetAttribute(attn_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)bw::KVLay::smem_bytes()) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tile_scores_big_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SCORES_BIG_SMEM) == cudaSuccess;
     ok &= cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)stc::kSmemBytes) == cudaSuccess;
     ok &= cudaFuncSetAttribute(head_stat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BUDGET_SMEM) ==
@@ -627,10 +624,6 @@ sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, cons
     return launch_status();
 }
 
-#ifndef SA_SCORES_TC
-#define SA_SCORES_TC 1
-#endif
-
 // Step 2 on the tensor cores (k_scores_tc.cuh): the pooled tables' tensor maps are encoded once
 // per call; each launch then covers rows [i0, i0 + rows) of heads h0 .. h0 + gz - 1.
 struct ScoreTcLaunch {
@@ -670,18 +663,6 @@ static sa_status score_tc_launch(ScoreTcLaunch* L, int64_t h0, int64_t i0, int64
     return launch_status();
 }
 
-// Large tile counts: 128 x 128 blocks (8 x 8 outputs per thread); small ones keep 64 x 64 blocks
-// so that enough CTAs fill the GPU.
-static void launch_scores(const ScoreArgs& a, unsigned gz, cudaStream_t stream) {
-    if (a.nt >= 1024 && a.rows >= 128) {
-        const dim3 grid((unsigned)((a.nt + 127) / 128), (unsigned)((a.rows + 127) / 128), gz);
-        tile_scores_big_kernel<<<grid, 256, SCORES_BIG_SMEM, stream>>>(a);
-    } else {
-        const dim3 grid((unsigned)((a.nt + 63) / 64), (unsigned)((a.rows + 63) / 64), gz);
-        tile_scores_kernel<<<grid, 256, 0, stream>>>(a);
-    }
-}
-
 sa_status sa_tile_scores(const sa_shape* shape, const float* q_pool, const float* k_pool, float* scores,
                          sa_stream_t stream) {
     Geo g;
@@ -690,24 +671,10 @@ sa_status sa_tile_scores(const sa_shape* shape, const float* q_pool, const float
     if (!q_pool || !k_pool || !scores || !aligned16(q_pool) || !aligned16(k_pool) || !aligned16(scores))
         return SA_ERR_INVALID_ARG;
     if (g.bh > 65535) return SA_ERR_UNSUPPORTED;
-    ScoreArgs a;
-    a.q_pool = q_pool;
-    a.k_pool = k_pool;
-    a.out = scores;
-    a.ldo = g.nt;
-    a.nt = (int32_t)g.nt;
-    a.h0 = 0;
-    a.i0 = 0;
-    a.rows = (int32_t)g.nt;
-    if ((g.nt + 63) / 64 > 65535) return SA_ERR_UNSUPPORTED;
     if ((st = ensure_attributes()) != SA_OK) return st;
-    if (SA_SCORES_TC) {
-        ScoreTcLaunch L;
-        if (!score_tc_prepare(&L, g, q_pool, k_pool, scores, g.nt)) return SA_ERR_CUDA;
-        return score_tc_launch(&L, 0, 0, g.nt, g.bh, stream);
-    }
-    launch_scores(a, (unsigned)g.bh, stream);
-    return launch_status();
+    ScoreTcLaunch L;
+    if (!score_tc_prepare(&L, g, q_pool, k_pool, scores, g.nt)) return SA_ERR_CUDA;
+    return score_tc_launch(&L, 0, 0, g.nt, g.bh, stream);
 }
 
 size_t sa_select_workspace_size(const sa_shape* shape, int32_t streamed) {
@@ -778,25 +745,11 @@ static sa_status select_impl(const sa_shape* shape, const float* scores_or_null,
     const int64_t R = (int64_t)select_rows_per_block(g);
     float* blk = static_cast<float*>(workspace_or_null);
     ScoreTcLaunch L;
-    if (SA_SCORES_TC && !score_tc_prepare(&L, g, q_pool, k_pool, blk, g.nt)) return SA_ERR_CUDA;
+    if (!score_tc_prepare(&L, g, q_pool, k_pool, blk, g.nt)) return SA_ERR_CUDA;
     for (int64_t h = 0; h < g.bh; ++h) {
         for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
             const int64_t rows = std::min<int64_t>(R, g.nt - i0);
-            if (SA_SCORES_TC) {
-                if ((st = score_tc_launch(&L, h, i0, rows, 1, stream)) != SA_OK) return st;
-            } else {
-                ScoreArgs sc;
-                sc.q_pool = q_pool;
-                sc.k_pool = k_pool;
-                sc.out = blk;
-                sc.ldo = g.nt;
-                sc.nt = (int32_t)g.nt;
-                sc.h0 = (int32_t)h;
-                sc.i0 = (int32_t)i0;
-                sc.rows = (int32_t)rows;
-                launch_scores(sc, 1u, stream);
-                if ((st = launch_status()) != SA_OK) return st;
-            }
+            if ((st = score_tc_launch(&L, h, i0, rows, 1, stream)) != SA_OK) return st;
             a.scores = blk;
             a.lds = g.nt;
             a.h0 = (int32_t)h;
@@ -852,25 +805,11 @@ sa_status sa_select_topk_noalloc(const sa_shape* shape, const float* q_pool, con
     a.k_head = nullptr;
     a.k_max = k;
     ScoreTcLaunch L;
-    if (SA_SCORES_TC && !score_tc_prepare(&L, g, q_pool, k_pool, blk, g.nt)) return SA_ERR_CUDA;
+    if (!score_tc_prepare(&L, g, q_pool, k_pool, blk, g.nt)) return SA_ERR_CUDA;
     for (int64_t h = 0; h < g.bh; ++h) {
         for (int64_t i0 = 0; i0 < g.nt; i0 += R) {
             const int64_t rows = std::min<int64_t>(R, g.nt - i0);
-            if (SA_SCORES_TC) {
-                if ((st = score_tc_launch(&L, h, i0, rows, 1, stream)) != SA_OK) return st;
-            } else {
-                ScoreArgs sc;
-                sc.q_pool = q_pool;
-                sc.k_pool = k_pool;
-                sc.out = blk;
-                sc.ldo = g.nt;
-                sc.nt = (int32_t)g.nt;
-                sc.h0 = (int32_t)h;
-                sc.i0 = (int32_t)i0;
-                sc.rows = (int32_t)rows;
-                launch_scores(sc, 1u, stream);
-                if ((st = launch_status()) != SA_OK) return st;
-            }
+            if ((st = score_tc_launch(&L, h, i0, rows, 1, stream)) != SA_OK) return st;
             a.scores = blk;
             a.lds = g.nt;
             a.h0 = (int32_t)h;
