@@ -983,13 +983,17 @@ def main(argv=None):
     ap.add_argument("--dense-budget", type=float, default=15.0,
                     help="seconds of timed dense-control calls (at least one call)")
     ap.add_argument("--frames", type=int, default=0,
-                    help="run the workload at another frame count, same tile sparsity (smaller profiling cases)")
+                    help="run the workload at another frame count, same budget k (smaller profiling cases)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with fewer heads, same shape per head (smaller profiling cases)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = BY_NAME[args.workload]
     if args.frames:
         w = with_frames(w, args.frames)
+    if args.heads:
+        w = w.scaled(name="%s_%dheads" % (w.name, args.heads), heads=args.heads)
     if args.impl == "reference":
         run_reference(args, w)
     elif args.sga:
