@@ -339,11 +339,21 @@ __device__ __forceinline__ uint32_t sel_find_bin(const uint32_t* hist, uint32_t 
                                                  SelBlockBin* out) {
     const int tid = threadIdx.x;
     uint32_t bins[BPT], lsum = 0;
+    if constexpr (BPT % 4 == 0) {  // 16-byte reads: a thread's bins are contiguous
 #pragma unroll
-    for (int u = 0; u < BPT; ++u) {
-        bins[u] = hist[BPT * tid + u];
-        lsum += bins[u];
+        for (int u = 0; u < BPT / 4; ++u) {
+            const uint4 b4 = reinterpret_cast<const uint4*>(hist + BPT * tid)[u];
+            bins[4 * u] = b4.x;
+            bins[4 * u + 1] = b4.y;
+            bins[4 * u + 2] = b4.z;
+            bins[4 * u + 3] = b4.w;
+        }
+    } else {
+#pragma unroll
+        for (int u = 0; u < BPT; ++u) bins[u] = hist[BPT * tid + u];
     }
+#pragma unroll
+    for (int u = 0; u < BPT; ++u) lsum += bins[u];
     uint32_t total;
     const uint32_t before = block_exclusive_scan(lsum, scratch, &total);
     const uint32_t want = min(want_in, total);
@@ -378,7 +388,7 @@ __device__ __forceinline__ bool select_row_block(const SelectArgs& a, int h, int
     uint16_t* lst = reinterpret_cast<uint16_t*>(hist1);
     uint32_t* selmask = hist1 + select_block_list_words(nt);  // [nwords]
     uint32_t* eqmask = selmask + nwords;                // [nwords]
-    __shared__ uint32_t hist2[SEL_BLOCK_H2];
+    __shared__ __align__(16) uint32_t hist2[SEL_BLOCK_H2];
     __shared__ uint32_t scratch[32];
     __shared__ __align__(8) uint64_t bar;
     __shared__ SelBlockBin sb;
@@ -423,14 +433,30 @@ __device__ __forceinline__ bool select_row_block(const SelectArgs& a, int h, int
         if (__syncthreads_or(!ok)) return false;  // timed out: the error word says so
     }
 
-    // ---- 1. keys in place + first-level histogram (sink slots taken out afterwards)
-    for (int c = tid; c < nt; c += SEL_BLOCK_THREADS) {
-        uint32_t key = 0u;
-        if (c < f0 || c >= f1) {
-            key = max(f32_order_key(__uint_as_float(keys[c])), 1u);
+    // ---- 1. keys in place + first-level histogram (sink slots taken out afterwards), four keys
+    // per 16-byte access over the aligned middle of the row
+    {
+        auto to_key = [&](int c, uint32_t bits) -> uint32_t {
+            if (c >= f0 && c < f1) return 0u;
+            const uint32_t key = max(f32_order_key(__uint_as_float(bits)), 1u);
             atomicAdd(&hist1[key >> 20], 1u);
+            return key;
+        };
+        const int va = min(nt, (int)((4u - mis) & 3u));  // keys + va is 16-byte aligned
+        const int vn = (nt - va) >> 2;
+        const int vb = va + 4 * vn;
+        if (tid < va) keys[tid] = to_key(tid, keys[tid]);
+        for (int g = tid; g < vn; g += SEL_BLOCK_THREADS) {
+            uint4* p = reinterpret_cast<uint4*>(keys + va) + g;
+            uint4 v = *p;
+            const int c = va + 4 * g;
+            v.x = to_key(c, v.x);
+            v.y = to_key(c + 1, v.y);
+            v.z = to_key(c + 2, v.z);
+            v.w = to_key(c + 3, v.w);
+            *p = v;
         }
-        keys[c] = key;
+        if (tid < nt - vb) keys[vb + tid] = to_key(vb + tid, keys[vb + tid]);
     }
     __syncthreads();
     if (s0 > 0) {  // slots below s0 hold sink rows only: not candidates
@@ -481,16 +507,35 @@ __device__ __forceinline__ bool select_row_block(const SelectArgs& a, int h, int
                 in_span = 1u << 20;
             }
         }
+        const bool vec = mis == 0u;  // keys 16-byte aligned: a word is eight 16-byte reads
         for (int wd = tid; wd < nwords; wd += SEL_BLOCK_THREADS) {
             uint32_t sm = 0u, im = 0u;
+            // past nt the reads land in the slack or the next region: masked below
+            if (vec) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int qq = (q + wd) & 7;  // rotated by the word: a quarter-warp reads 8 bank groups
+                    const uint4 k4 = reinterpret_cast<const uint4*>(keys + wd * 32)[qq];
+                    const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t key = kv[u];
+                        const uint32_t sbit = (!sel_none && key >= sel_from && key != 0u) ? 1u : 0u;
+                        const uint32_t ibit = (key != 0u && key - in_lo < in_span) ? 1u : 0u;
+                        sm |= sbit << (4 * qq + u);
+                        im |= ibit << (4 * qq + u);
+                    }
+                }
+            } else {
 #pragma unroll 8
-            for (int j = 0; j < 32; ++j) {
-                const int jj = (j + wd) & 31;
-                const uint32_t key = keys[wd * 32 + jj];  // past nt: slack or the next region, masked below
-                const uint32_t sbit = (!sel_none && key >= sel_from && key != 0u) ? 1u : 0u;
-                const uint32_t ibit = (key != 0u && key - in_lo < in_span) ? 1u : 0u;
-                sm |= sbit << jj;
-                im |= ibit << jj;
+                for (int j = 0; j < 32; ++j) {
+                    const int jj = (j + wd) & 31;
+                    const uint32_t key = keys[wd * 32 + jj];
+                    const uint32_t sbit = (!sel_none && key >= sel_from && key != 0u) ? 1u : 0u;
+                    const uint32_t ibit = (key != 0u && key - in_lo < in_span) ? 1u : 0u;
+                    sm |= sbit << jj;
+                    im |= ibit << jj;
+                }
             }
             const int rem = nt - wd * 32;  // valid tiles in this word
             const uint32_t valid = rem >= 32 ? 0xFFFFFFFFu : ((1u << rem) - 1u);
