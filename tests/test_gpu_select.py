@@ -8,8 +8,9 @@ one first-level bin), huge and tiny magnitudes, all negative, and two strided fa
 tile (from tile 3) far above the rest, or far below it, which would mislead any selection that
 estimated the threshold from a strided sample of the row.  Signed zeros are avoided: the
 oracle treats -0 and +0 as equal, the kernel orders -0 below +0 (both are valid top-k sets).
-Shapes cover the warp-per-row kernel (rows up to 2048 tiles) and the block-per-row kernel
-(longer rows), with and without whole sink slots.
+Shapes cover the warp-per-row kernel (rows up to 2048 tiles; under 16 words of 32 tiles one tile per lane,
+above one 32-tile word per lane) and the block-per-row kernel (longer rows), with and without
+whole sink slots.
 """
 import numpy as np
 import pytest
@@ -52,7 +53,9 @@ def score_rows(bh, nt, seed):
 
 
 @pytest.mark.parametrize("frames,tokens,tile,n_sink,k,bh", [
-    (40, 700, 128, 5, 17, 2),       # 240 tiles: warp-per-row kernel
+    (40, 700, 128, 5, 17, 2),       # 240 tiles: warp-per-row kernel, one tile per lane
+    (120, 1374, 128, 5, 130, 2),    # 1320 tiles: warp kernel, one 32-tile word per lane
+    (100, 1374, 128, 256, 40, 1),   # 1100 tiles: the same with two whole sink slots per frame
     (7, 300, 64, 0, 3, 3),          # ragged frames, tile 64
     (5, 1374, 128, 0, 60, 1),       # k above the candidate count: every candidate kept
     (200, 1374, 128, 5, 130, 2),    # 2200 tiles: block-per-row kernel

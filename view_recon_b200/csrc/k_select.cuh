@@ -28,6 +28,7 @@
 #define SEL_H1 1024        // first level: key bits 31..22
 #define SEL_H2 256         // refinement digits: bits 21..14, 13..6, 5..0
 #define SEL_LCAP 256       // boundary-bin keys gathered for refinement (more: refined from the row)
+#define SEL_WORD_MIN_WORDS 16  // rows of at least this many 32-tile words: word-per-lane gather and emission
 #define SEL_SMEM_BUDGET (44 * 1024)  // per CTA: small CTAs of few rows keep ~20 warps per SM resident
 
 struct SelectArgs {
@@ -116,6 +117,54 @@ __device__ __forceinline__ SelBin sel_find_bin_warp(const uint32_t* hist, uint32
     return r;
 }
 
+__device__ __forceinline__ uint32_t sel_warp_inclusive_scan(uint32_t v, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += y;
+    }
+    return v;
+}
+
+// Masks of the 32-tile word w of a staged row of keys (bit j: tile 32 w + j; tiles past nt and
+// of the own frame [f0, f1) excluded from .y, the own frame always set in .x):
+//   .x  selected: key >= sel_from (candidates only, key >= 1), unless sel_none
+//   .y  in range: key - lo < span (candidates only)
+// The reads start at element `rot` mod 32 (16-byte chunk rot mod 8 when vec), so that lanes
+// reading different words hit different banks; past nt they land in the slack or the next
+// region of the warp's shared memory and are masked.
+__device__ __forceinline__ uint2 sel_word_mask(const uint32_t* keys, int w, int nt, int f0, int f1, uint32_t sel_from,
+                                               bool sel_none, uint32_t lo, uint32_t span, bool vec, int rot) {
+    uint32_t sm = 0u, im = 0u;
+    if (vec) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int qq = (q + rot) & 7;
+            const uint4 k4 = reinterpret_cast<const uint4*>(keys + w * 32)[qq];
+            const uint32_t kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t key = kv[u];
+                sm |= ((!sel_none && key >= sel_from && key != 0u) ? 1u : 0u) << (4 * qq + u);
+                im |= ((key != 0u && key - lo < span) ? 1u : 0u) << (4 * qq + u);
+            }
+        }
+    } else {
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+            const int jj = (j + rot) & 31;
+            const uint32_t key = keys[w * 32 + jj];
+            sm |= ((!sel_none && key >= sel_from && key != 0u) ? 1u : 0u) << jj;
+            im |= ((key != 0u && key - lo < span) ? 1u : 0u) << jj;
+        }
+    }
+    const int rem = nt - w * 32;
+    const uint32_t valid = rem >= 32 ? 0xFFFFFFFFu : ((1u << rem) - 1u);
+    const int lo_b = min(max(f0 - 32 * w, 0), 32), hi_b = min(max(f1 - 32 * w, 0), 32);
+    const uint32_t own = (hi_b == 32 ? 0xFFFFFFFFu : ((1u << hi_b) - 1u)) & ~(lo_b == 32 ? 0xFFFFFFFFu : ((1u << lo_b) - 1u));
+    return make_uint2((sm & valid) | own, im & valid & ~own);
+}
+
 __global__ void __launch_bounds__(32 * SEL_MAX_WARPS) select_topk_warp_kernel(SelectArgs a) {
     extern __shared__ __align__(16) uint32_t sel_smem[];
     __shared__ __align__(8) uint64_t bars[SEL_MAX_WARPS];
@@ -124,6 +173,7 @@ __global__ void __launch_bounds__(32 * SEL_MAX_WARPS) select_topk_warp_kernel(Se
     const int x = blockIdx.x * nw + warp;  // local row
     if (x >= a.rows) return;               // no CTA-wide synchronisation follows
     const int nt = a.nt;
+    const int nwords = (nt + 31) >> 5;
     uint32_t* stage = sel_smem + (size_t)warp * select_warp_words(nt);
     uint32_t* hist = stage + select_stage_words(nt);  // [SEL_H1]
     uint32_t* lkeys = hist + SEL_H1;                  // [SEL_LCAP]
@@ -217,16 +267,36 @@ __global__ void __launch_bounds__(32 * SEL_MAX_WARPS) select_topk_warp_kernel(Se
 
     if (!whole && kk > 0) {
         // ---- 2. gather the keys of the boundary bin (all of them land in the list unless
-        // there are more than SEL_LCAP; then the refinement reads them from the row)
+        // there are more than SEL_LCAP; then the refinement reads them from the row).  Long
+        // rows: lane l takes the 32-tile words l, l + 32, ...; a word's mask is built in
+        // registers, a warp scan places its keys
         uint32_t m = 0;
-        for (int c0 = 0; c0 < nt; c0 += 32) {
-            const int c = c0 + lane;
-            const uint32_t key = c < nt ? keys[c] : 0u;
-            const bool in = key != 0u && (key >> 22) == prefix;
-            const uint32_t bi = __ballot_sync(0xffffffffu, in);
-            const uint32_t pos = m + __popc(bi & ((1u << lane) - 1u));
-            if (in && pos < SEL_LCAP) lkeys[pos] = key;
-            m += __popc(bi);
+        if (nwords >= SEL_WORD_MIN_WORDS) {
+            const uint32_t bin_lo = prefix << 22;  // the bin is [bin_lo, bin_lo + 2^22)
+            for (int r0 = 0; r0 < nwords; r0 += 32) {
+                const int w = r0 + lane;
+                const uint32_t im = w < nwords ? sel_word_mask(keys, w, nt, f0, f1, 0xFFFFFFFFu, true, bin_lo,
+                                                               1u << 22, mis == 0u, lane).y
+                                               : 0u;
+                const uint32_t cnt = __popc(im);
+                const uint32_t inc = sel_warp_inclusive_scan(cnt, lane);
+                uint32_t pos2 = m + inc - cnt;
+                for (uint32_t e = im; e; e &= e - 1u) {
+                    if (pos2 < SEL_LCAP) lkeys[pos2] = keys[w * 32 + __ffs(e) - 1];
+                    ++pos2;
+                }
+                m += __shfl_sync(0xffffffffu, inc, 31);
+            }
+        } else {  // short rows: one tile per lane and ballots
+            for (int c0 = 0; c0 < nt; c0 += 32) {
+                const int c = c0 + lane;
+                const uint32_t key = c < nt ? keys[c] : 0u;
+                const bool in = key != 0u && (key >> 22) == prefix;
+                const uint32_t bi = __ballot_sync(0xffffffffu, in);
+                const uint32_t pos = m + __popc(bi & ((1u << lane) - 1u));
+                if (in && pos < SEL_LCAP) lkeys[pos] = key;
+                m += __popc(bi);
+            }
         }
         __syncwarp();
         const bool from_list = m <= SEL_LCAP;
@@ -254,26 +324,64 @@ __global__ void __launch_bounds__(32 * SEL_MAX_WARPS) select_topk_warp_kernel(Se
         }
     }
 
-    // ---- 4. emit the kept tiles in ascending order
+    // ---- 4. emit the kept tiles in ascending order: own frame, keys above the threshold,
+    // and the first `need` keys at it in index order; for long rows word by word, lane l
+    // taking words l, l + 32, ... of each round, warp scans placing the ties and the output
     int32_t* out = a.kept_idx + ((int64_t)h * nt + i) * a.max_kept;
     uint32_t pos = 0, tie_before = 0;
-    for (int c0 = 0; c0 < nt; c0 += 32) {
-        const int c = c0 + lane;
-        const uint32_t key = c < nt ? keys[c] : 0u;
-        const uint32_t p = key >> shift;
-        const bool own = c >= f0 && c < f1;
-        const bool above = key != 0u && (p > prefix || (whole && p == prefix));
-        const bool tie = !whole && key != 0u && p == prefix;
-        bool sel = own || above;
-        const uint32_t bt = __ballot_sync(0xffffffffu, tie);
-        if (bt) {
-            sel = sel || (tie && tie_before + __popc(bt & ((1u << lane) - 1u)) < need);
-            tie_before += __popc(bt);
+    if (nwords >= SEL_WORD_MIN_WORDS) {
+        const uint64_t lo64 = (uint64_t)prefix << shift, hi64 = ((uint64_t)prefix + 1ull) << shift;
+        const uint64_t from64 = whole ? lo64 : hi64;
+        const bool sel_none = from64 > 0xFFFFFFFFull;
+        const uint32_t sel_from = sel_none ? 0xFFFFFFFFu : max((uint32_t)from64, 1u);
+        const bool ties = !whole && need > 0 && lo64 <= 0xFFFFFFFFull;
+        const uint32_t t_lo = ties ? (uint32_t)lo64 : 0u;
+        const uint32_t t_span = ties ? (uint32_t)(hi64 - lo64) : 0u;  // shift <= 22: span <= 2^22
+        for (int r0 = 0; r0 < nwords; r0 += 32) {
+            const int w = r0 + lane;
+            uint2 mk = make_uint2(0u, 0u);
+            if (w < nwords) mk = sel_word_mask(keys, w, nt, f0, f1, sel_from, sel_none, t_lo, t_span, mis == 0u, lane);
+            uint32_t sm = mk.x, tm = mk.y;
+            const uint32_t tc = __popc(tm);
+            const uint32_t tinc = sel_warp_inclusive_scan(tc, lane);
+            const uint32_t tb = tie_before + tinc - tc;  // ties in earlier words
+            if (tm && tb < need) {
+                const uint32_t take = min(tc, need - tb);
+                for (uint32_t t = 0; t < take; ++t) {
+                    const uint32_t low = tm & (0u - tm);
+                    sm |= low;
+                    tm ^= low;
+                }
+            }
+            tie_before += __shfl_sync(0xffffffffu, tinc, 31);
+            const uint32_t sc = __popc(sm);
+            const uint32_t sinc = sel_warp_inclusive_scan(sc, lane);
+            uint32_t o = pos + sinc - sc;
+            for (uint32_t e = sm; e; e &= e - 1u) {
+                if (o < (uint32_t)a.max_kept) out[o] = w * 32 + __ffs(e) - 1;
+                ++o;
+            }
+            pos += __shfl_sync(0xffffffffu, sinc, 31);
         }
-        const uint32_t bs = __ballot_sync(0xffffffffu, sel);
-        const uint32_t o = pos + __popc(bs & ((1u << lane) - 1u));
-        if (sel && o < (uint32_t)a.max_kept) out[o] = c;
-        pos += __popc(bs);
+    } else {  // short rows: one tile per lane and ballots
+        for (int c0 = 0; c0 < nt; c0 += 32) {
+            const int c = c0 + lane;
+            const uint32_t key = c < nt ? keys[c] : 0u;
+            const uint32_t p = key >> shift;
+            const bool own = c >= f0 && c < f1;
+            const bool above = key != 0u && (p > prefix || (whole && p == prefix));
+            const bool tie = !whole && key != 0u && p == prefix;
+            bool sel = own || above;
+            const uint32_t bt = __ballot_sync(0xffffffffu, tie);
+            if (bt) {
+                sel = sel || (tie && tie_before + __popc(bt & ((1u << lane) - 1u)) < need);
+                tie_before += __popc(bt);
+            }
+            const uint32_t bs = __ballot_sync(0xffffffffu, sel);
+            const uint32_t o = pos + __popc(bs & ((1u << lane) - 1u));
+            if (sel && o < (uint32_t)a.max_kept) out[o] = c;
+            pos += __popc(bs);
+        }
     }
     uint32_t tot = pos;
     if (tot > (uint32_t)a.max_kept) {
