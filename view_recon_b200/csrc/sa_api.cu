@@ -88,6 +88,7 @@ sa_status launch_status() {
 std::mutex g_attr_mu;
 bool g_attr_done[kMaxDevices];
 bool g_tc_regs_ok[kMaxDevices];
+int g_sm_count[kMaxDevices];  // SMs per device, read once with the attributes
 
 sa_status ensure_attributes() {
     int dev = 0;
@@ -124,6 +125,12 @@ sa_status ensure_attributes() {
         return SA_ERR_CUDA;
     }
     g_tc_regs_ok[dev] = (uint32_t)fa.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    g_sm_count[dev] = sms;
     g_attr_done[dev] = true;
     return SA_OK;
 }
@@ -628,11 +635,15 @@ sa_status sa_tile_pool(const sa_shape* shape, const void* q, const void* k, cons
 // per call; each launch then covers rows [i0, i0 + rows) of heads h0 .. h0 + gz - 1.
 struct ScoreTcLaunch {
     ScoreTcArgs a;
+    int32_t sms;  // SMs of the current device
 };
 
 static bool score_tc_prepare(ScoreTcLaunch* L, const Geo& g, const float* q_pool, const float* k_pool, float* out,
                              int64_t ldo) {
     memset(&L->a, 0, sizeof(L->a));
+    int dev = 0;  // ensure_attributes() has run: the SM count is known
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices || g_sm_count[dev] < 1) return false;
+    L->sms = g_sm_count[dev];
     if (!encode_rows_e(&L->a.tm_q, q_pool, g.bh * g.nt, false, 128) ||
         !encode_rows_e(&L->a.tm_k, k_pool, g.bh * g.nt, false, 128))
         return false;
@@ -653,10 +664,11 @@ static sa_status score_tc_launch(ScoreTcLaunch* L, int64_t h0, int64_t i0, int64
     const int64_t gy = (rows + 127) / 128;
     if (gy > 65535 || gz > 65535 || gy < 1 || gz < 1) return SA_ERR_UNSUPPORTED;
     // One CTA per SM at a time (211 KB of shared memory): with fewer row tiles than SMs the chunks
-    // of a row tile are split so that the grid is one wave of at most 148 CTAs; otherwise every
-    // CTA takes whole row tiles.
+    // of a row tile are split so that the grid is one wave of at most one CTA per SM; otherwise
+    // every CTA takes whole row tiles.
+    const int64_t sms = L->sms;
     const int64_t tiles = gy * gz;
-    const int64_t per_tile = tiles >= 148 ? 1 : 148 / tiles;
+    const int64_t per_tile = tiles >= sms ? 1 : sms / tiles;
     a.chunks_per_cta = (int32_t)((a.n_chunks + per_tile - 1) / per_tile);
     const int64_t gx = (a.n_chunks + a.chunks_per_cta - 1) / a.chunks_per_cta;
     score_tc_kernel<<<dim3((unsigned)gx, (unsigned)gy, (unsigned)gz), 384, stc::kSmemBytes, stream>>>(a);
