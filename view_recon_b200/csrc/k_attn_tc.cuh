@@ -225,7 +225,8 @@ struct TcLayout {
     // per slot: q_full, kv_full[S], kv_empty[S], s_full, s_free, p_full, pv_done, drain
     static constexpr int kBarsPerSlot = 6 + 2 * STAGES;
     static constexpr int kMisc = kBars + 8 * kBarsPerSlot * NSLOT;  // tmem base, abort flag
-    static constexpr int kEnd = kMisc + 16;
+    static constexpr int kMeta = kMisc + 16;  // [slot][stage] the item's {kind, lo, hi, chunk}
+    static constexpr int kEnd = kMeta + NSLOT * STAGES * 16;
     static constexpr uint32_t colS(int x) { return x * 128; }
     static constexpr uint32_t colP(int x) { return NSLOT * 128 + x * 64; }
     static constexpr uint32_t colO(int x) { return NSLOT * 128 + NSLOT * 64 + x * 64; }
@@ -257,6 +258,9 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
     uint64_t* p_full = s_free + 1;
     uint64_t* pv_done = p_full + 1;
     uint64_t* drain_bar = pv_done + 1;
+    // what the softmax needs of each item, written by the producer before it arms the stage's
+    // kv_full barrier (whose completion the softmax observes before reading it)
+    int4* meta = reinterpret_cast<int4*>(smem + Lay::kMeta) + x * STAGES;
 
     if (threadIdx.x == 0) {
         uint64_t* all = reinterpret_cast<uint64_t*>(smem + Lay::kBars);
@@ -315,10 +319,12 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                 const int j_cur = win.entry(a, sl, n, lane);
                 if (leader) {
                     const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
+                    if (it.kind < 0) sa_flag_error(SA_ERR_BAD_LIST);  // skipped list entry
                     const CUtensorMap* mk = it.kind == 1 ? &a.tm_sk : (it.kind == 2 ? &a.tm_lk : &a.tm_k);
                     const CUtensorMap* mv = it.kind == 1 ? &a.tm_svt : (it.kind == 2 ? &a.tm_lvt : &a.tm_vt);
                     uint8_t* dk = sKV + s * 2 * tc::kTileBytes;
-                    mbar_arrive_expect_tx(&kv_full[s], 2 * tc::kTileBytes);
+                    meta[s] = make_int4(it.kind, it.lo, it.hi, it.chunk);
+                    mbar_arrive_expect_tx(&kv_full[s], 2 * tc::kTileBytes);  // releases meta[s]
                     tma_load_2d(dk, mk, &kv_full[s], 0, it.krow);
                     tma_load_2d(dk + tc::kTileBytes, mv, &kv_full[s], 0, it.vrow);
                     tma_load_2d(dk + tc::kTileBytes + tc::kTileBytes / 2, mv, &kv_full[s], 64, it.vrow);
@@ -388,7 +394,6 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
     } else {
         // ------------------------------------------------------------------ softmax group
         setmaxnreg_inc<Lay::kRegsSoftmax>();
-        const int st = threadIdx.x - 128 - 128 * x;  // 0..127
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -398,11 +403,18 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
         int lm_ptr = 0;                                              // landmark chunks: list cursor
-        tc::ListWindow win(a, sl, lane);
         for (int n = 0; n < sl.n_items; ++n) {
-            const int j_cur = win.entry(a, sl, n, lane);
-            const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
-            if (it.kind < 0 && st == 0) sa_flag_error(SA_ERR_BAD_LIST);  // skipped list entry
+            // the item's kind and valid columns, as the producer decoded them: its stage has
+            // landed (S(n) was computed from it), so this wait returns at once and orders the read
+            if (!mbar_wait_warp(&kv_full[n % STAGES], (n / STAGES) & 1u, abort_flag)) { ok = false; break; }
+            tc::Item it;
+            {
+                const int4 md = meta[n % STAGES];
+                it.kind = md.x;
+                it.lo = md.y;
+                it.hi = md.z;
+                it.chunk = md.w;
+            }
             if (!mbar_wait_warp(s_full, n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint32_t sv[128];
