@@ -233,7 +233,9 @@ struct TcLayout {
     static size_t smem_bytes() { return 1024 + kEnd; }
 };
 
-template <int NSLOT, int STAGES>
+// LANDMARK: the call has landmark chunks (a.landmark); without them the softmax carries no
+// landmark code, which leaves it more registers.
+template <int NSLOT, int STAGES, bool LANDMARK>
 __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __grid_constant__ TcArgs a) {
     using Lay = TcLayout<NSLOT, STAGES>;
     static_assert(NSLOT == 2, "warp roles are laid out for two slots");
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             // Masked columns become -inf; landmark chunks add their per-column bias in base-2
             // units (so their values are scaled here and `mul` becomes 1).
             float mul = a.scale_log2;
-            if (it.kind == 2) {
+            if (LANDMARK && it.kind == 2) {
                 // listed tiles of this chunk: the next run of the ascending list
                 uint32_t mw[4] = {0u, 0u, 0u, 0u};
                 const int c_lo = it.chunk * 128;

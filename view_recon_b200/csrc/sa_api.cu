@@ -97,7 +97,9 @@ sa_status ensure_attributes() {
     std::lock_guard<std::mutex> lk(g_attr_mu);
     if (g_attr_done[dev]) return SA_OK;
     bool ok = true;
-    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStages, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(attn_tcg_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)tcg::Cfg<false>::smem_bytes()) == cudaSuccess;
@@ -118,13 +120,16 @@ sa_status ensure_attributes() {
     // The tensor-core kernel moves registers between its warpgroups (setmaxnreg); that is only
     // satisfiable if the block is launched with at least the registers the split hands out.
     cudaFuncAttributes fa;
-    ok &= cudaFuncGetAttributes(&fa, attn_tc_kernel<kTcSlots, kTcStages>) == cudaSuccess;
+    cudaFuncAttributes fa_lm;
+    ok &= cudaFuncGetAttributes(&fa, attn_tc_kernel<kTcSlots, kTcStages, false>) == cudaSuccess;
+    ok &= cudaFuncGetAttributes(&fa_lm, attn_tc_kernel<kTcSlots, kTcStages, true>) == cudaSuccess;
     using Lay = TcLayout<kTcSlots, kTcStages>;
     if (!ok) {
         cudaGetLastError();
         return SA_ERR_CUDA;
     }
-    g_tc_regs_ok[dev] = (uint32_t)fa.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded;
+    g_tc_regs_ok[dev] = (uint32_t)fa.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded &&
+                        (uint32_t)fa_lm.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
         cudaGetLastError();
@@ -406,7 +411,10 @@ sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v,
         const size_t smem = Lay::smem_bytes();
         if (smem > 227 * 1024) return SA_ERR_UNSUPPORTED;
         const int grid = (a.total_items + kTcSlots - 1) / kTcSlots;
-        attn_tc_kernel<kTcSlots, kTcStages><<<grid, Lay::kThreads, smem, stream>>>(a);
+        if (a.landmark)
+            attn_tc_kernel<kTcSlots, kTcStages, true><<<grid, Lay::kThreads, smem, stream>>>(a);
+        else
+            attn_tc_kernel<kTcSlots, kTcStages, false><<<grid, Lay::kThreads, smem, stream>>>(a);
         return launch_status();
     }
     {
