@@ -17,10 +17,13 @@
 //                   (128-byte swizzle);
 //   warps 1, 3      tcgen05.mma issuers of slots 0, 1 (one elected lane; warp 1 also owns
 //                   the TMEM allocation):
-//                     S_x = Q_x K^T   (M=128, N=128, K=64; A and B K-major in shared memory)
+//                     S_x = Q_x K^T   (M=128, N=128, K=64; A and B K-major in shared memory),
+//                     plus, for an item with key columns outside its valid range [lo, hi),
+//                     S_x += 1 . bias^T (one K=16 step; bias -2^100 on those columns, 0
+//                     elsewhere, written by the producer) so that the softmax needs no mask;
 //                     O_x += P_x V    (M=128, N=64, K=128; P read from TMEM, V^T K-major);
 //   warpgroup 1+x   the softmax group of slot x; thread r owns row r: tcgen05.ld of its 128
-//                   scores, masking, base-2 online softmax with a lazy max (O is rescaled
+//                   scores, base-2 online softmax with a lazy max (O is rescaled
 //                   only when the row max grows by more than 2^8), P written back to TMEM
 //                   as bf16, O rescale in TMEM, final normalisation.
 // TMEM columns per slot: S 128 (f32), P 64 (bf16 pairs), O 64 (f32): 512 in total.
@@ -211,7 +214,7 @@ __device__ __forceinline__ bool elect_one() {
 
 }  // namespace tc
 
-template <int NSLOT, int STAGES>
+template <int NSLOT, int STAGES, bool BIAS>
 struct TcLayout {
     static constexpr int kThreads = 128 + 128 * NSLOT;
     static constexpr uint32_t kTmemCols = 512;
@@ -221,7 +224,11 @@ struct TcLayout {
     static constexpr uint32_t kRegsNeeded = 128 * kRegsControl + 128 * NSLOT * kRegsSoftmax;
     static constexpr int kQ = 0;
     static constexpr int kKV = NSLOT * tc::kTileBytes;                 // [slot][stage] K + V^T
-    static constexpr int kBars = kKV + NSLOT * STAGES * 2 * tc::kTileBytes;
+    // BIAS: the mask operands, a tile of ones (A) and, at the four 16-column K steps of one
+    // more tile, the column-bias operand (B) of each [slot][stage]
+    static constexpr int kOnes = kKV + NSLOT * STAGES * 2 * tc::kTileBytes;
+    static constexpr int kBias = kOnes + (BIAS ? tc::kTileBytes : 0);
+    static constexpr int kBars = kBias + (BIAS ? tc::kTileBytes : 0);
     // per slot: q_full, kv_full[S], kv_empty[S], s_full, s_free, p_full, pv_done, drain
     static constexpr int kBarsPerSlot = 6 + 2 * STAGES;
     static constexpr int kMisc = kBars + 8 * kBarsPerSlot * NSLOT;  // tmem base, abort flag
@@ -235,11 +242,14 @@ struct TcLayout {
 
 // LANDMARK: the call has landmark chunks (a.landmark); without them the softmax carries no
 // landmark code, which leaves it more registers.
-template <int NSLOT, int STAGES, bool LANDMARK>
+// BIAS: key columns outside an item's valid range are masked by the bias product on the tensor
+// cores (the ring then has room for at most four stages); otherwise the softmax masks them.
+template <int NSLOT, int STAGES, bool LANDMARK, bool BIAS>
 __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __grid_constant__ TcArgs a) {
-    using Lay = TcLayout<NSLOT, STAGES>;
+    using Lay = TcLayout<NSLOT, STAGES, BIAS>;
     static_assert(NSLOT == 2, "warp roles are laid out for two slots");
     static_assert(NSLOT * (128 + 64 + 64) <= 512, "TMEM columns");
+    static_assert(!BIAS || NSLOT * STAGES <= 4, "one 16-column K step of the bias tile per ring stage");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
@@ -260,8 +270,9 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
     uint64_t* p_full = s_free + 1;
     uint64_t* pv_done = p_full + 1;
     uint64_t* drain_bar = pv_done + 1;
-    // what the softmax needs of each item, written by the producer before it arms the stage's
-    // kv_full barrier (whose completion the softmax observes before reading it)
+    // each item's {kind, lo, hi, chunk}, written by the producer before it arms the stage's
+    // kv_full barrier, whose completion the MMA issuer (and, in landmark calls, the softmax)
+    // observes before reading it
     int4* meta = reinterpret_cast<int4*>(smem + Lay::kMeta) + x * STAGES;
 
     if (threadIdx.x == 0) {
@@ -281,6 +292,14 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
         }
         *abort_flag = 0;
         fence_barrier_init();
+    }
+    if (BIAS) {
+        // every bf16 element of the ones tile is 1.0, so each of its 16-column K steps is the
+        // all-ones A operand of the mask product, whatever the swizzle
+        uint4* ones = reinterpret_cast<uint4*>(smem + Lay::kOnes);
+        const uint4 v = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+        for (int i = threadIdx.x; i < tc::kTileBytes / 16; i += Lay::kThreads) ones[i] = v;
+        fence_proxy_async_smem();
     }
     if ((warp == 0 || warp == 2) && lane == 0) {
         tma_prefetch_desc(&a.tm_q);
@@ -319,14 +338,32 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                     break;
                 }
                 const int j_cur = win.entry(a, sl, n, lane);
+                const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
+                if (BIAS && (it.lo > 0 || it.hi < 128)) {
+                    // The item's column bias, B operand of one more product S += ones . bias^T:
+                    // row r (key column r) holds sixteen bf16 elements of -2^96 when r is outside
+                    // [lo, hi), so that S there becomes -2^100, and zeros otherwise, which leave
+                    // S unchanged.  The stage's K step q sits in the 16-byte chunks 2q, 2q + 1
+                    // of each 128-byte row, stored at chunk ^ (r & 7) (128-byte swizzle).
+                    const int q = x * STAGES + (int)s;
+                    uint8_t* bias = smem + Lay::kBias;
+                    for (int r = lane; r < 128; r += 32) {
+                        const uint32_t w = (r < it.lo || r >= it.hi) ? 0xEF80EF80u : 0u;
+                        const uint4 v = make_uint4(w, w, w, w);
+                        *reinterpret_cast<uint4*>(bias + r * 128 + (((2 * q) ^ (r & 7)) << 4)) = v;
+                        *reinterpret_cast<uint4*>(bias + r * 128 + (((2 * q + 1) ^ (r & 7)) << 4)) = v;
+                    }
+                    fence_proxy_async_smem();  // the MMA reads it through the async proxy
+                }
+                __syncwarp();
                 if (leader) {
-                    const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
                     if (it.kind < 0) sa_flag_error(SA_ERR_BAD_LIST);  // skipped list entry
                     const CUtensorMap* mk = it.kind == 1 ? &a.tm_sk : (it.kind == 2 ? &a.tm_lk : &a.tm_k);
                     const CUtensorMap* mv = it.kind == 1 ? &a.tm_svt : (it.kind == 2 ? &a.tm_lvt : &a.tm_vt);
                     uint8_t* dk = sKV + s * 2 * tc::kTileBytes;
                     meta[s] = make_int4(it.kind, it.lo, it.hi, it.chunk);
-                    mbar_arrive_expect_tx(&kv_full[s], 2 * tc::kTileBytes);  // releases meta[s]
+                    // releases meta[s] and the warp's bias rows
+                    mbar_arrive_expect_tx(&kv_full[s], 2 * tc::kTileBytes);
                     tma_load_2d(dk, mk, &kv_full[s], 0, it.krow);
                     tma_load_2d(dk + tc::kTileBytes, mv, &kv_full[s], 0, it.vrow);
                     tma_load_2d(dk + tc::kTileBytes + tc::kTileBytes / 2, mv, &kv_full[s], 64, it.vrow);
@@ -348,6 +385,8 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t dk0 = smem_desc_sw128(smem_u32(sKV), 16, 1024);
             const uint64_t dv0 = smem_desc_sw128(smem_u32(sKV + tc::kTileBytes), 16, 1024);
+            const uint64_t d_ones = smem_desc_sw128(smem_u32(smem + Lay::kOnes), 16, 1024);
+            const uint64_t d_bias = smem_desc_sw128(smem_u32(smem + Lay::kBias), 16, 1024) + 2 * (x * STAGES);
             constexpr uint64_t kStageStep = (2 * tc::kTileBytes) >> 4;
             // S(n) is issued as soon as its tile has landed and the softmax has read S(n-1),
             // P.V(n-1) right after it, as soon as P(n-1) is in TMEM
@@ -362,6 +401,10 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             umma_ss(tmem + Lay::colS(x), dq + 2 * kk, dk + 2 * kk, tc::kIdescS, kk > 0);
+                        // columns outside [lo, hi): add the bias the producer wrote for this stage
+                        const int4 md = meta[s];
+                        if (BIAS && (md.y > 0 || md.z < 128))
+                            umma_ss(tmem + Lay::colS(x), d_ones, d_bias + 2 * s, tc::kIdescS, 1);
                         umma_commit(s_full);
                     }
                     __syncwarp();
@@ -406,16 +449,17 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
         bool ok = true;
         int lm_ptr = 0;                                              // landmark chunks: list cursor
         for (int n = 0; n < sl.n_items; ++n) {
-            // the item's kind and valid columns, as the producer decoded them: its stage has
-            // landed (S(n) was computed from it), so this wait returns at once and orders the read
-            if (!mbar_wait_warp(&kv_full[n % STAGES], (n / STAGES) & 1u, abort_flag)) { ok = false; break; }
-            tc::Item it;
-            {
+            // the item's kind, valid columns and chunk, as the producer decoded them (landmark
+            // calls and softmax masking only); its stage has landed (S(n) was computed from it),
+            // so this wait returns at once and orders the read
+            int kind = 0, lo = 0, hi = 128, chunk = 0;
+            if (LANDMARK || !BIAS) {
+                if (!mbar_wait_warp(&kv_full[n % STAGES], (n / STAGES) & 1u, abort_flag)) { ok = false; break; }
                 const int4 md = meta[n % STAGES];
-                it.kind = md.x;
-                it.lo = md.y;
-                it.hi = md.z;
-                it.chunk = md.w;
+                kind = md.x;
+                lo = md.y;
+                hi = md.z;
+                chunk = md.w;
             }
             if (!mbar_wait_warp(s_full, n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
@@ -432,13 +476,14 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             tc_fence_before();
             mbar_arrive(s_free);
 
-            // Masked columns become -inf; landmark chunks add their per-column bias in base-2
-            // units (so their values are scaled here and `mul` becomes 1).
+            // Key columns outside an item's valid range arrive as -2^100 (BIAS: the bias product)
+            // or are set to -inf here; landmark chunks add their per-column bias in base-2 units
+            // (so their values are scaled here and `mul` becomes 1) and mask their listed tiles.
             float mul = a.scale_log2;
-            if (LANDMARK && it.kind == 2) {
+            if (LANDMARK && kind == 2) {
                 // listed tiles of this chunk: the next run of the ascending list
                 uint32_t mw[4] = {0u, 0u, 0u, 0u};
-                const int c_lo = it.chunk * 128;
+                const int c_lo = chunk * 128;
                 while (lm_ptr < sl.cnt) {
                     const int j = __ldg(sl.list + lm_ptr);
                     if (j >= c_lo + 128) break;
@@ -460,11 +505,11 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                     }
                 }
                 mul = 1.0f;
-            } else if (it.lo > 0 || it.hi < 128) {
+            } else if (!BIAS && (lo > 0 || hi < 128)) {
                 // valid columns [lo, hi) as four 32-bit words; one bit test and select per column
 #pragma unroll
                 for (int w4 = 0; w4 < 4; ++w4) {
-                    const int b0 = min(max(it.lo - 32 * w4, 0), 32), b1 = min(max(it.hi - 32 * w4, 0), 32);
+                    const int b0 = min(max(lo - 32 * w4, 0), 32), b1 = min(max(hi - 32 * w4, 0), 32);
                     const uint32_t below_hi = b1 == 32 ? 0xFFFFFFFFu : ((1u << b1) - 1u);
                     const uint32_t below_lo = b0 == 32 ? 0xFFFFFFFFu : ((1u << b0) - 1u);
                     const uint32_t valid = below_hi & ~below_lo;

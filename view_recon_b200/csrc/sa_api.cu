@@ -25,7 +25,8 @@ static __device__ __align__(256) float g_sa_noalloc_scores[kNoallocScratchFloats
 namespace {
 
 constexpr int kTcSlots = 2;
-constexpr int kTcStages = 3;  // per slot
+constexpr int kTcStages = 2;       // per slot, sparse calls: the mask operands take the third stage's room
+constexpr int kTcStagesDense = 3;  // per slot, dense calls: one partial tile per head, masked in the softmax
 constexpr int kMaxDevices = 64;
 
 struct Geo {
@@ -97,10 +98,12 @@ sa_status ensure_attributes() {
     std::lock_guard<std::mutex> lk(g_attr_mu);
     if (g_attr_done[dev]) return SA_OK;
     bool ok = true;
-    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStages, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               227 * 1024) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStages, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStages, true, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(attn_tc_kernel<kTcSlots, kTcStagesDense, false, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(attn_tcg_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)tcg::Cfg<false>::smem_bytes()) == cudaSuccess;
     ok &= cudaFuncSetAttribute(attn_tcg_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -119,17 +122,18 @@ sa_status ensure_attributes() {
                                (int)select_block_smem_bytes(SEL_MAX_NT)) == cudaSuccess;
     // The tensor-core kernel moves registers between its warpgroups (setmaxnreg); that is only
     // satisfiable if the block is launched with at least the registers the split hands out.
-    cudaFuncAttributes fa;
-    cudaFuncAttributes fa_lm;
-    ok &= cudaFuncGetAttributes(&fa, attn_tc_kernel<kTcSlots, kTcStages, false>) == cudaSuccess;
-    ok &= cudaFuncGetAttributes(&fa_lm, attn_tc_kernel<kTcSlots, kTcStages, true>) == cudaSuccess;
-    using Lay = TcLayout<kTcSlots, kTcStages>;
+    cudaFuncAttributes fa, fa_lm, fa_d;
+    ok &= cudaFuncGetAttributes(&fa, attn_tc_kernel<kTcSlots, kTcStages, false, true>) == cudaSuccess;
+    ok &= cudaFuncGetAttributes(&fa_lm, attn_tc_kernel<kTcSlots, kTcStages, true, true>) == cudaSuccess;
+    ok &= cudaFuncGetAttributes(&fa_d, attn_tc_kernel<kTcSlots, kTcStagesDense, false, false>) == cudaSuccess;
+    using Lay = TcLayout<kTcSlots, kTcStages, true>;  // the register split is the same in all three
     if (!ok) {
         cudaGetLastError();
         return SA_ERR_CUDA;
     }
     g_tc_regs_ok[dev] = (uint32_t)fa.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded &&
-                        (uint32_t)fa_lm.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded;
+                        (uint32_t)fa_lm.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded &&
+                        (uint32_t)fa_d.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
         cudaGetLastError();
@@ -394,7 +398,8 @@ sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v,
         a.q_per_head = dense ? (int32_t)((g.L + 127) / 128) : (int32_t)g.nt;
         a.total_items = (int32_t)(g.bh * a.q_per_head);
         a.scale_log2 = (float)((double)g.scale * 1.4426950408889634);
-        using Lay = TcLayout<kTcSlots, kTcStages>;
+        using Lay = TcLayout<kTcSlots, kTcStages, true>;
+        using LayD = TcLayout<kTcSlots, kTcStagesDense, false>;
         {
             int dev = 0;
             if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
@@ -408,13 +413,15 @@ sa_status attn_common(const Geo& g, const void* q, const void* k, const void* v,
             for (int64_t j = 0; j < g.nt; ++j)
                 if ((int64_t)(((uint64_t)j * a.tpf_magic) >> 32) != j / g.tpf) return SA_ERR_UNSUPPORTED;
         }
-        const size_t smem = Lay::smem_bytes();
+        const size_t smem = dense ? LayD::smem_bytes() : Lay::smem_bytes();
         if (smem > 227 * 1024) return SA_ERR_UNSUPPORTED;
         const int grid = (a.total_items + kTcSlots - 1) / kTcSlots;
-        if (a.landmark)
-            attn_tc_kernel<kTcSlots, kTcStages, true><<<grid, Lay::kThreads, smem, stream>>>(a);
+        if (dense)
+            attn_tc_kernel<kTcSlots, kTcStagesDense, false, false><<<grid, Lay::kThreads, smem, stream>>>(a);
+        else if (a.landmark)
+            attn_tc_kernel<kTcSlots, kTcStages, true, true><<<grid, Lay::kThreads, smem, stream>>>(a);
         else
-            attn_tc_kernel<kTcSlots, kTcStages, false><<<grid, Lay::kThreads, smem, stream>>>(a);
+            attn_tc_kernel<kTcSlots, kTcStages, false, true><<<grid, Lay::kThreads, smem, stream>>>(a);
         return launch_status();
     }
     {
