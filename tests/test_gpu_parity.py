@@ -36,6 +36,9 @@ CASES = [
     small("streamed_select", frames=4, tokens=600, k=3, streamed=True),
     small("window_landmark_streamed", frames=6, tokens=500, k=4, landmark=True, streamed=True, window=2),
     small("one_tile_per_frame", frames=6, tokens=100, k=2, landmark=True),
+    # 130 special tokens: every frame's first key tile has no key row (own frame, listed first, so
+    # a query tile's first item is masked whole) and its second starts at column 2
+    small("sinks_fill_a_tile", frames=3, tokens=400, n_sink=130, k=2),
 ]
 
 
