@@ -240,13 +240,14 @@ struct TcLayout {
     static size_t smem_bytes() { return 1024 + kEnd; }
 };
 
-// LANDMARK: the call has landmark chunks (a.landmark); without them the softmax carries no
-// landmark code, which leaves it more registers.
+// LANDMARK: the call has landmark chunks (a.landmark): the producer also writes their bias
+// (multiplicity terms, listed tiles masked); without them it carries no landmark code.
 // BIAS: key columns outside an item's valid range are masked by the bias product on the tensor
 // cores (the ring then has room for at most four stages); otherwise the softmax masks them.
 template <int NSLOT, int STAGES, bool LANDMARK, bool BIAS>
 __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __grid_constant__ TcArgs a) {
     using Lay = TcLayout<NSLOT, STAGES, BIAS>;
+    static_assert(BIAS || !LANDMARK, "landmark chunks take their bias through the bias product");
     static_assert(NSLOT == 2, "warp roles are laid out for two slots");
     static_assert(NSLOT * (128 + 64 + 64) <= 512, "TMEM columns");
     static_assert(!BIAS || NSLOT * STAGES <= 4, "one 16-column K step of the bias tile per ring stage");
@@ -271,7 +272,7 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
     uint64_t* pv_done = p_full + 1;
     uint64_t* drain_bar = pv_done + 1;
     // each item's {kind, lo, hi, chunk}, written by the producer before it arms the stage's
-    // kv_full barrier, whose completion the MMA issuer (and, in landmark calls, the softmax)
+    // kv_full barrier, whose completion the MMA issuer (and, masking in the softmax, the softmax)
     // observes before reading it
     int4* meta = reinterpret_cast<int4*>(smem + Lay::kMeta) + x * STAGES;
 
@@ -331,6 +332,7 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                 tma_load_2d(sQ, &a.tm_q, q_full, 0, sl.qrow);
             }
             tc::ListWindow win(a, sl, lane);
+            int lm_ptr = 0;  // landmark chunks: list cursor (warp-uniform)
             for (int n = 0; n < n_items; ++n) {
                 const uint32_t s = n % STAGES, ph = (n / STAGES) & 1u;
                 if (!mbar_wait_warp(&kv_empty[s], ph ^ 1u, abort_flag)) {
@@ -339,19 +341,63 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                 }
                 const int j_cur = win.entry(a, sl, n, lane);
                 const tc::Item it = tc::get_item_j(a, sl, n, j_cur);
-                if (BIAS && (it.lo > 0 || it.hi < 128)) {
-                    // The item's column bias, B operand of one more product S += ones . bias^T:
-                    // row r (key column r) holds sixteen bf16 elements of -2^96 when r is outside
-                    // [lo, hi), so that S there becomes -2^100, and zeros otherwise, which leave
-                    // S unchanged.  The stage's K step q sits in the 16-byte chunks 2q, 2q + 1
-                    // of each 128-byte row, stored at chunk ^ (r & 7) (128-byte swizzle).
+                const bool lm_item = LANDMARK && it.kind == 2;
+                if (BIAS && (lm_item || it.lo > 0 || it.hi < 128)) {
+                    // The item's column bias, B operand of one more product S += ones . bias^T
+                    // (every element of the A tile is 1, so row r of the bias, key column r, adds
+                    // the sum of its sixteen bf16 elements to column r of S).  The stage's K step q
+                    // sits in the 16-byte chunks 2q, 2q + 1 of each 128-byte row, stored at
+                    // chunk ^ (r & 7) (128-byte swizzle).
                     const int q = x * STAGES + (int)s;
                     uint8_t* bias = smem + Lay::kBias;
-                    for (int r = lane; r < 128; r += 32) {
-                        const uint32_t w = (r < it.lo || r >= it.hi) ? 0xEF80EF80u : 0u;
-                        const uint4 v = make_uint4(w, w, w, w);
-                        *reinterpret_cast<uint4*>(bias + r * 128 + (((2 * q) ^ (r & 7)) << 4)) = v;
-                        *reinterpret_cast<uint4*>(bias + r * 128 + (((2 * q + 1) ^ (r & 7)) << 4)) = v;
+                    if (!lm_item) {
+                        // key columns outside [lo, hi): sixteen elements of -2^96, so that S there
+                        // becomes -2^100; zeros elsewhere leave S unchanged
+                        for (int r = lane; r < 128; r += 32) {
+                            const uint32_t w = (r < it.lo || r >= it.hi) ? 0xEF80EF80u : 0u;
+                            const uint4 v = make_uint4(w, w, w, w);
+                            *reinterpret_cast<uint4*>(bias + r * 128 + (((2 * q) ^ (r & 7)) << 4)) = v;
+                            *reinterpret_cast<uint4*>(bias + r * 128 + (((2 * q + 1) ^ (r & 7)) << 4)) = v;
+                        }
+                    } else {
+                        // landmark chunk: the listed tiles of the chunk (the next run of the
+                        // ascending list, 32 entries per step) get -2^100, the others their
+                        // multiplicity term log2(c_j) in units of S (divided by the base-2 scale),
+                        // split into three bf16 parts so that their sum keeps f32 accuracy
+                        const int c_lo = it.chunk * 128;
+                        uint32_t mw[4] = {0u, 0u, 0u, 0u};
+                        for (;;) {
+                            const int e = lm_ptr + lane;
+                            const int j = e < sl.cnt ? __ldg(sl.list + e) : 0x7FFFFFFF;
+                            const bool here = j >= c_lo && j < c_lo + 128;
+#pragma unroll
+                            for (int w4 = 0; w4 < 4; ++w4)
+                                mw[w4] |= __reduce_or_sync(0xffffffffu,
+                                                           (here && ((j - c_lo) >> 5) == w4) ? 1u << (j & 31) : 0u);
+                            const int used = __popc(__ballot_sync(0xffffffffu, j < c_lo + 128));
+                            lm_ptr += used;
+                            if (used < 32) break;
+                        }
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4) {
+                            const int r = 32 * w4 + lane;
+                            const float b2 = __ldg(a.lbias2 + c_lo + r);  // log2 c_j, or -inf
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (((mw[w4] >> lane) & 1u) || !(b2 > -INFINITY)) {
+                                v.x = 0xF180u;  // -2^100
+                            } else {
+                                const float b = __fdiv_rn(b2, a.scale_log2);
+                                const __nv_bfloat16 p0 = __float2bfloat16_rn(b);
+                                const float r1 = b - __bfloat162float(p0);
+                                const __nv_bfloat16 p1 = __float2bfloat16_rn(r1);
+                                const __nv_bfloat16 p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+                                v.x = (uint32_t)__bfloat16_as_ushort(p0) | ((uint32_t)__bfloat16_as_ushort(p1) << 16);
+                                v.y = (uint32_t)__bfloat16_as_ushort(p2);
+                            }
+                            *reinterpret_cast<uint4*>(bias + r * 128 + (((2 * q) ^ (r & 7)) << 4)) = v;
+                            *reinterpret_cast<uint4*>(bias + r * 128 + (((2 * q + 1) ^ (r & 7)) << 4)) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
                     }
                     fence_proxy_async_smem();  // the MMA reads it through the async proxy
                 }
@@ -401,9 +447,9 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             umma_ss(tmem + Lay::colS(x), dq + 2 * kk, dk + 2 * kk, tc::kIdescS, kk > 0);
-                        // columns outside [lo, hi): add the bias the producer wrote for this stage
+                        // columns outside [lo, hi), landmark chunks: add the bias the producer wrote
                         const int4 md = meta[s];
-                        if (BIAS && (md.y > 0 || md.z < 128))
+                        if (BIAS && ((LANDMARK && md.x == 2) || md.y > 0 || md.z < 128))
                             umma_ss(tmem + Lay::colS(x), d_ones, d_bias + 2 * s, tc::kIdescS, 1);
                         umma_commit(s_full);
                     }
@@ -447,19 +493,16 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
         const uint32_t tO = tmem + Lay::colO(x) + lane_off;
         float m_run = -INFINITY, l_run = 0.0f;
         bool ok = true;
-        int lm_ptr = 0;                                              // landmark chunks: list cursor
         for (int n = 0; n < sl.n_items; ++n) {
-            // the item's kind, valid columns and chunk, as the producer decoded them (landmark
-            // calls and softmax masking only); its stage has landed (S(n) was computed from it),
-            // so this wait returns at once and orders the read
-            int kind = 0, lo = 0, hi = 128, chunk = 0;
-            if (LANDMARK || !BIAS) {
+            // softmax masking only: the item's valid columns, as the producer decoded them; its
+            // stage has landed (S(n) was computed from it), so this wait returns at once and
+            // orders the read
+            int lo = 0, hi = 128;
+            if (!BIAS) {
                 if (!mbar_wait_warp(&kv_full[n % STAGES], (n / STAGES) & 1u, abort_flag)) { ok = false; break; }
                 const int4 md = meta[n % STAGES];
-                kind = md.x;
                 lo = md.y;
                 hi = md.z;
-                chunk = md.w;
             }
             if (!mbar_wait_warp(s_full, n & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
@@ -476,36 +519,11 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
             tc_fence_before();
             mbar_arrive(s_free);
 
-            // Key columns outside an item's valid range arrive as -2^100 (BIAS: the bias product)
-            // or are set to -inf here; landmark chunks add their per-column bias in base-2 units
-            // (so their values are scaled here and `mul` becomes 1) and mask their listed tiles.
-            float mul = a.scale_log2;
-            if (LANDMARK && kind == 2) {
-                // listed tiles of this chunk: the next run of the ascending list
-                uint32_t mw[4] = {0u, 0u, 0u, 0u};
-                const int c_lo = chunk * 128;
-                while (lm_ptr < sl.cnt) {
-                    const int j = __ldg(sl.list + lm_ptr);
-                    if (j >= c_lo + 128) break;
-                    if (j >= c_lo) mw[(j - c_lo) >> 5] |= 1u << (j & 31);
-                    ++lm_ptr;
-                }
-                const float4* bp = reinterpret_cast<const float4*>(a.lbias2 + c_lo);
-#pragma unroll
-                for (int c4 = 0; c4 < 32; ++c4) {
-                    const float4 bv = __ldg(bp + c4);
-                    const uint32_t word = mw[c4 >> 3];
-                    const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c = 4 * c4 + u;
-                        const bool listed = (word >> (c & 31)) & 1u;
-                        const float xv = fmaf(__uint_as_float(sv[c]), a.scale_log2, bb[u]);
-                        sv[c] = __float_as_uint(listed ? -INFINITY : xv);
-                    }
-                }
-                mul = 1.0f;
-            } else if (!BIAS && (lo > 0 || hi < 128)) {
+            // Key columns outside an item's valid range and listed tiles of a landmark chunk arrive
+            // as -2^100, landmark chunks with their multiplicity term added (BIAS: the bias
+            // product); without BIAS the invalid columns are set to -inf here.
+            const float mul = a.scale_log2;
+            if (!BIAS && (lo > 0 || hi < 128)) {
                 // valid columns [lo, hi) as four 32-bit words; one bit test and select per column
 #pragma unroll
                 for (int w4 = 0; w4 < 4; ++w4) {
