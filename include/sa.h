@@ -241,6 +241,9 @@ size_t sa_sparse_attn_workspace_size(const sa_shape* shape, int32_t landmark);
  * O has the shape's dtype, [bh][S*N][d]; lse is f32 [bh][S*N].  Products run on the tensor
  * cores with f32 accumulation and an f32 softmax: bf16 operands for bf16 inputs (landmark means
  * enter rounded to bf16), tf32 operands (each f32 rounded to the nearest tf32) for f32 inputs.
+ * With bf16 tile-128 inputs the masks of partial tiles and listed landmark tiles (-2^100) and
+ * the landmark terms b_t (divided by scale, as three bf16 parts: about f32 accuracy) are added
+ * to the scores by one more tensor-core product.
  * Lists must be ascending with entries in [0, nt) and no repeats; a list from sa_select_topk
  * always is.  Entries beyond kept_cnt are ignored.  An out-of-range entry is skipped and
  * reported as SA_ERR_BAD_LIST by sa_check_device_error.
