@@ -55,9 +55,13 @@ struct __align__(64) TcArgs {
 };
 
 // Of every 8 column pairs of a score row, this many take their exponentials on the FMA pipe
-// (exp2_poly2) and the rest on the MUFU (ex2.approx).
+// (exp2_poly2) and the rest on the MUFU (ex2.approx): sparse launches (no mask code in the
+// softmax) and dense launches (masks in the softmax) were each timed with 0 to 3.
 #ifndef SA_EXP2_FMA_PAIRS_PER8
-#define SA_EXP2_FMA_PAIRS_PER8 2
+#define SA_EXP2_FMA_PAIRS_PER8 1
+#endif
+#ifndef SA_EXP2_FMA_PAIRS_PER8_DENSE
+#define SA_EXP2_FMA_PAIRS_PER8_DENSE 2
 #endif
 
 namespace tc {
@@ -218,9 +222,10 @@ template <int NSLOT, int STAGES, bool BIAS>
 struct TcLayout {
     static constexpr int kThreads = 128 + 128 * NSLOT;
     static constexpr uint32_t kTmemCols = 512;
-    // registers per thread after the split: warpgroup 0 gives, the softmax groups take
-    static constexpr uint32_t kRegsControl = 40;
-    static constexpr uint32_t kRegsSoftmax = 232;
+    // registers per thread after the split: warpgroup 0 gives, the softmax groups take (the
+    // producer's bias writes want a few more control registers in sparse launches)
+    static constexpr uint32_t kRegsControl = BIAS ? 48 : 40;
+    static constexpr uint32_t kRegsSoftmax = BIAS ? 224 : 232;
     static constexpr uint32_t kRegsNeeded = 128 * kRegsControl + 128 * NSLOT * kRegsSoftmax;
     static constexpr int kQ = 0;
     static constexpr int kKV = NSLOT * tc::kTileBytes;                 // [slot][stage] K + V^T
@@ -561,7 +566,7 @@ __global__ void __launch_bounds__(128 + 128 * NSLOT, 1) attn_tc_kernel(const __g
                 const float2 xv =
                     __ffma2_rn(make_float2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), mul2, neg2);
                 float2 p;
-                if ((c & 7) >= 8 - SA_EXP2_FMA_PAIRS_PER8) {
+                if ((c & 7) >= 8 - (BIAS ? SA_EXP2_FMA_PAIRS_PER8 : SA_EXP2_FMA_PAIRS_PER8_DENSE)) {
                     p = exp2_poly2(xv);  // FMA pipe: takes load off the MUFU
                 } else {
                     p.x = ex2_approx(xv.x);

@@ -126,14 +126,15 @@ sa_status ensure_attributes() {
     ok &= cudaFuncGetAttributes(&fa, attn_tc_kernel<kTcSlots, kTcStages, false, true>) == cudaSuccess;
     ok &= cudaFuncGetAttributes(&fa_lm, attn_tc_kernel<kTcSlots, kTcStages, true, true>) == cudaSuccess;
     ok &= cudaFuncGetAttributes(&fa_d, attn_tc_kernel<kTcSlots, kTcStagesDense, false, false>) == cudaSuccess;
-    using Lay = TcLayout<kTcSlots, kTcStages, true>;  // the register split is the same in all three
+    using Lay = TcLayout<kTcSlots, kTcStages, true>;
+    using LayD = TcLayout<kTcSlots, kTcStagesDense, false>;
     if (!ok) {
         cudaGetLastError();
         return SA_ERR_CUDA;
     }
     g_tc_regs_ok[dev] = (uint32_t)fa.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded &&
                         (uint32_t)fa_lm.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded &&
-                        (uint32_t)fa_d.numRegs * (uint32_t)Lay::kThreads >= Lay::kRegsNeeded;
+                        (uint32_t)fa_d.numRegs * (uint32_t)LayD::kThreads >= LayD::kRegsNeeded;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
         cudaGetLastError();
